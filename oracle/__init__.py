@@ -1,0 +1,139 @@
+"""fp64 CPU oracle for grouped-query attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+legs of ``bench.py`` may import this package.  The CUDA library never calls
+it, and it shares no code with the CUDA library: the arithmetic lives in
+``gqa_oracle.c`` (plain C, fp64, full score matrix per (batch, head)); this
+file only compiles it with gcc, loads it with ctypes and marshals arrays.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` to facts the
+pages and the mathematics fix (closed forms, invariants, a brute-force
+restatement through the expand-then-reshape K/V repetition, the KV-cache
+worked number).  Parity status: pinned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gqa_oracle.c")
+_LIB = os.path.join(_HERE, "libgqa_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_int = ctypes.c_int
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle (plain gcc, IEEE fp64, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-pthread", "-fno-fast-math",
+                               "-ffp-contract=off", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.oracle_prefill.argtypes = [_u16p, _u16p, _u16p, _f64p] + [_int] * 7 + [ctypes.c_double, _int]
+            lib.oracle_prefill_rows.argtypes = ([_u16p, _u16p, _u16p, _f64p] + [_int] * 7 +
+                                                [ctypes.c_double, _i32p, _int, _int])
+            lib.oracle_decode.argtypes = [_u16p, _u16p, _u16p, _i32p, _f64p] + [_int] * 4 + [ctypes.c_double, _int]
+            lib.oracle_prefill_probs.argtypes = ([_u16p, _u16p, _u16p, _f64p] + [_int] * 7 +
+                                                 [ctypes.c_double, _int, _int])
+            for f in (lib.oracle_prefill, lib.oracle_prefill_rows, lib.oracle_decode, lib.oracle_prefill_probs):
+                f.restype = _int
+            _lib = lib
+    return _lib
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 bit patterns from a torch bf16 tensor or a uint16 array."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch
+    assert x.dtype == torch.bfloat16, x.dtype
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def _p(a, t):
+    return a.ctypes.data_as(t)
+
+
+def prefill(q, k, v, causal: bool = True, scale: float | None = None, n_threads: int = 0) -> np.ndarray:
+    """Exact attention for q [B,S_q,h,d], k/v [B,S_kv,n_kv,d]; returns fp64 [B,S_q,h,d]."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, S_q, h, d = qb.shape
+    _, S_kv, n_kv, _ = kb.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.empty((B, S_q, h, d), dtype=np.float64)
+    rc = _load().oracle_prefill(_p(qb, _u16p), _p(kb, _u16p), _p(vb, _u16p), _p(out, _f64p),
+                                B, S_q, S_kv, h, n_kv, d, int(bool(causal)), float(scale), n_threads)
+    if rc:
+        raise ValueError("oracle_prefill rejected its arguments")
+    return out
+
+
+def prefill_rows(q, k, v, sample, causal: bool = True, scale: float | None = None,
+                 n_threads: int = 0) -> np.ndarray:
+    """Output rows for the (b, i, r) triplets in ``sample`` ([n,3] int); returns fp64 [n,d]."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, S_q, h, d = qb.shape
+    _, S_kv, n_kv, _ = kb.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    s = np.ascontiguousarray(np.asarray(sample, dtype=np.int32).reshape(-1, 3))
+    out = np.empty((s.shape[0], d), dtype=np.float64)
+    rc = _load().oracle_prefill_rows(_p(qb, _u16p), _p(kb, _u16p), _p(vb, _u16p), _p(out, _f64p),
+                                     B, S_q, S_kv, h, n_kv, d, int(bool(causal)), float(scale),
+                                     _p(s, _i32p), s.shape[0], n_threads)
+    if rc:
+        raise ValueError("oracle_prefill_rows rejected its arguments")
+    return out
+
+
+def decode(q, k_cache, v_cache, seqlens, scale: float | None = None, n_threads: int = 0) -> np.ndarray:
+    """One decode step: q [B,h,d], packed caches [T,n_kv,d], seqlens [B]; returns fp64 [B,h,d]."""
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    B, h, d = qb.shape
+    n_kv = kb.shape[1]
+    lens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32).reshape(B))
+    if int(np.clip(lens, 0, None).sum()) > kb.shape[0]:
+        raise ValueError("seqlens exceed the cache rows")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.empty((B, h, d), dtype=np.float64)
+    rc = _load().oracle_decode(_p(qb, _u16p), _p(kb, _u16p), _p(vb, _u16p), _p(lens, _i32p),
+                               _p(out, _f64p), B, h, n_kv, d, float(scale), n_threads)
+    if rc:
+        raise ValueError("oracle_decode rejected its arguments")
+    return out
+
+
+def prefill_probs(q, k, v, b: int, i: int, causal: bool = True, scale: float | None = None) -> np.ndarray:
+    """The S_q x S_kv softmax matrix of unit (b, i)."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, S_q, h, d = qb.shape
+    _, S_kv, n_kv, _ = kb.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    probs = np.empty((S_q, S_kv), dtype=np.float64)
+    rc = _load().oracle_prefill_probs(_p(qb, _u16p), _p(kb, _u16p), _p(vb, _u16p), _p(probs, _f64p),
+                                      B, S_q, S_kv, h, n_kv, d, int(bool(causal)), float(scale), b, i)
+    if rc:
+        raise ValueError("oracle_prefill_probs rejected its arguments")
+    return probs

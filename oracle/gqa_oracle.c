@@ -1,0 +1,285 @@
+/*
+ * Plain fp64 CPU oracle for grouped-query attention.  TEST INFRASTRUCTURE ONLY:
+ * only the tests, the smoke check and the bench's CPU-baseline leg may load it.
+ * It shares no code, header or constant with the CUDA library.
+ *
+ * What it computes (the plain definition, written out):
+ *   "Evolution of AI Attention Mechanisms" (toolsku), section "MHA Mathematical
+ *   Formulation": per head, Attn = softmax(Q K^T * scale) V, heads being
+ *   contiguous d_h slices of the hidden dimension;
+ *   same page, "GQA Implementation": with n_rep = h / n_kv, K/V head g is
+ *   repeated n_rep times (expand then reshape), so query head i reads KV
+ *   head i / n_rep;
+ *   same page, "MHA Implementation": masked scores are set to -inf before the
+ *   softmax, and past K/V are concatenated in front of the new ones (so new
+ *   queries are the LAST S_q positions: bottom-right causal alignment);
+ *   "Attention variants" (saadho), "What this topic covers": FlashAttention
+ *   computes this same exact result, so the oracle is the untiled definition.
+ *
+ * For every (batch b, query head i) the full score matrix of the requested
+ * query rows against all keys is materialised in fp64, masked, soft-maxed row
+ * by row (max subtracted, as a softmax is usually evaluated), and multiplied
+ * by V.  Inputs are bf16 bit patterns; each is widened exactly to fp64.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+static double bf16_value(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/*
+ * One attention unit.  q_rows: nr query vectors (length d, already fp64).
+ * keys/vals: row j of K and V for j < nk, given as bf16 pointers with a row
+ * stride in elements.  visible[r]: query row r sees keys j < visible[r].
+ * out: nr x d.  probs (optional): nr x nk softmax matrix.
+ */
+static int attend(const double *q_rows, int nr, const uint16_t *k0, const uint16_t *v0,
+                  long kv_row_stride, int nk, int d, const int *visible, double scale,
+                  double *out, double *probs) {
+    double *S = (double *)malloc(sizeof(double) * (size_t)(nr > 0 ? nr : 1) * (size_t)(nk > 0 ? nk : 1));
+    double *kd = (double *)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1) * (size_t)d);
+    double *vd = (double *)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1) * (size_t)d);
+    if (!S || !kd || !vd) { free(S); free(kd); free(vd); return -1; }
+    for (int j = 0; j < nk; ++j)
+        for (int c = 0; c < d; ++c) {
+            kd[(size_t)j * d + c] = bf16_value(k0[(size_t)j * kv_row_stride + c]);
+            vd[(size_t)j * d + c] = bf16_value(v0[(size_t)j * kv_row_stride + c]);
+        }
+    /* scores, with the mask */
+    for (int r = 0; r < nr; ++r)
+        for (int j = 0; j < nk; ++j) {
+            double *s = &S[(size_t)r * nk + j];
+            if (j >= visible[r]) { *s = -INFINITY; continue; }
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) acc += q_rows[(size_t)r * d + c] * kd[(size_t)j * d + c];
+            *s = acc * scale;
+        }
+    /* row softmax, then P V */
+    for (int r = 0; r < nr; ++r) {
+        double *srow = &S[(size_t)r * nk];
+        double *orow = &out[(size_t)r * d];
+        for (int c = 0; c < d; ++c) orow[c] = 0.0;
+        if (visible[r] <= 0) {            /* no key: the row is defined as zero */
+            if (probs) for (int j = 0; j < nk; ++j) probs[(size_t)r * nk + j] = 0.0;
+            continue;
+        }
+        double m = -INFINITY;
+        for (int j = 0; j < nk; ++j) if (srow[j] > m) m = srow[j];
+        double sum = 0.0;
+        for (int j = 0; j < nk; ++j) {
+            srow[j] = (srow[j] == -INFINITY) ? 0.0 : exp(srow[j] - m);
+            sum += srow[j];
+        }
+        for (int j = 0; j < nk; ++j) srow[j] /= sum;
+        if (probs) memcpy(&probs[(size_t)r * nk], srow, sizeof(double) * (size_t)nk);
+        for (int j = 0; j < nk; ++j) {
+            double p = srow[j];
+            if (p == 0.0) continue;
+            for (int c = 0; c < d; ++c) orow[c] += p * vd[(size_t)j * d + c];
+        }
+    }
+    free(S); free(kd); free(vd);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* thread pool over units                                                    */
+
+typedef struct {
+    int kind;                 /* 0 prefill, 1 decode */
+    const uint16_t *q, *k, *v;
+    const int32_t *seqlens;
+    const long *offsets;      /* decode: first cache row of each sequence */
+    double *out;
+    int B, S_q, S_kv, h, n_kv, d, causal;
+    double scale;
+    /* sampled prefill rows: triplets (b, i, r); NULL = every row */
+    const int32_t *sample;
+    int n_sample;
+    int n_units;
+    int n_threads;
+    int failed;
+} job_t;
+
+typedef struct { job_t *job; int tid; } worker_arg_t;
+
+static void run_prefill_unit(job_t *J, int b, int i, const int *rows, int nr, double *out_rows) {
+    int G = J->h / J->n_kv;
+    int g = i / G;                                  /* the group of query head i */
+    int d = J->d;
+    double *qd = (double *)malloc(sizeof(double) * (size_t)nr * d);
+    int *vis = (int *)malloc(sizeof(int) * (size_t)nr);
+    if (!qd || !vis) { free(qd); free(vis); J->failed = 1; return; }
+    for (int t = 0; t < nr; ++t) {
+        int r = rows[t];
+        const uint16_t *qrow = J->q + (((size_t)b * J->S_q + r) * J->h + i) * d;
+        for (int c = 0; c < d; ++c) qd[(size_t)t * d + c] = bf16_value(qrow[c]);
+        int lim = J->S_kv;
+        if (J->causal) {
+            int last = r + (J->S_kv - J->S_q);   /* bottom-right alignment */
+            if (last + 1 < lim) lim = last + 1;
+            if (lim < 0) lim = 0;
+        }
+        vis[t] = lim;
+    }
+    const uint16_t *k0 = J->k + ((size_t)b * J->S_kv * J->n_kv + g) * d;
+    const uint16_t *v0 = J->v + ((size_t)b * J->S_kv * J->n_kv + g) * d;
+    if (attend(qd, nr, k0, v0, (long)J->n_kv * d, J->S_kv, d, vis, J->scale, out_rows, NULL))
+        J->failed = 1;
+    free(qd); free(vis);
+}
+
+static void run_decode_unit(job_t *J, int b, int i) {
+    int G = J->h / J->n_kv;
+    int g = i / G;
+    int d = J->d;
+    int L = J->seqlens[b];
+    double *orow = J->out + ((size_t)b * J->h + i) * d;
+    if (L <= 0) { for (int c = 0; c < d; ++c) orow[c] = 0.0; return; }
+    double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!qd) { J->failed = 1; return; }
+    const uint16_t *qrow = J->q + ((size_t)b * J->h + i) * d;
+    for (int c = 0; c < d; ++c) qd[c] = bf16_value(qrow[c]);
+    const uint16_t *k0 = J->k + ((size_t)J->offsets[b] * J->n_kv + g) * d;
+    const uint16_t *v0 = J->v + ((size_t)J->offsets[b] * J->n_kv + g) * d;
+    int vis = L;
+    if (attend(qd, 1, k0, v0, (long)J->n_kv * d, L, d, &vis, J->scale, orow, NULL)) J->failed = 1;
+    free(qd);
+}
+
+static void *worker(void *p) {
+    worker_arg_t *a = (worker_arg_t *)p;
+    job_t *J = a->job;
+    for (int u = a->tid; u < J->n_units; u += J->n_threads) {
+        if (J->kind == 1) {
+            run_decode_unit(J, u / J->h, u % J->h);
+        } else if (J->sample) {
+            const int32_t *s = J->sample + 3 * (size_t)u;
+            int r = s[2];
+            run_prefill_unit(J, s[0], s[1], &r, 1, J->out + (size_t)u * J->d);
+        } else {
+            int b = u / J->h, i = u % J->h;
+            int *rows = (int *)malloc(sizeof(int) * (size_t)J->S_q);
+            double *tmp = (double *)malloc(sizeof(double) * (size_t)J->S_q * J->d);
+            if (!rows || !tmp) { free(rows); free(tmp); J->failed = 1; continue; }
+            for (int r = 0; r < J->S_q; ++r) rows[r] = r;
+            run_prefill_unit(J, b, i, rows, J->S_q, tmp);
+            /* scatter to out[b, r, i, :] */
+            for (int r = 0; r < J->S_q; ++r)
+                memcpy(J->out + (((size_t)b * J->S_q + r) * J->h + i) * J->d,
+                       tmp + (size_t)r * J->d, sizeof(double) * (size_t)J->d);
+            free(rows); free(tmp);
+        }
+    }
+    return NULL;
+}
+
+static int run_job(job_t *J, int n_threads) {
+    if (n_threads <= 0) n_threads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > J->n_units) n_threads = J->n_units > 0 ? J->n_units : 1;
+    J->n_threads = n_threads;
+    J->failed = 0;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)n_threads);
+    worker_arg_t *args = (worker_arg_t *)malloc(sizeof(worker_arg_t) * (size_t)n_threads);
+    if (!th || !args) { free(th); free(args); return -1; }
+    for (int t = 0; t < n_threads; ++t) {
+        args[t].job = J; args[t].tid = t;
+        pthread_create(&th[t], NULL, worker, &args[t]);
+    }
+    for (int t = 0; t < n_threads; ++t) pthread_join(th[t], NULL);
+    free(th); free(args);
+    return J->failed ? -1 : 0;
+}
+
+static int check_shape(int B, int h, int n_kv, int d) {
+    return B > 0 && h > 0 && n_kv > 0 && d > 0 && h % n_kv == 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* exported entry points                                                     */
+
+/* Causal or full prefill.  q [B,S_q,h,d], k/v [B,S_kv,n_kv,d] bf16 bits,
+ * out [B,S_q,h,d] fp64.  Returns 0, or -1 on bad arguments / no memory. */
+int oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *out,
+                   int B, int S_q, int S_kv, int h, int n_kv, int d, int causal,
+                   double scale, int n_threads) {
+    if (!check_shape(B, h, n_kv, d) || S_q <= 0 || S_kv <= 0) return -1;
+    job_t J = {0};
+    J.kind = 0; J.q = q; J.k = k; J.v = v; J.out = out;
+    J.B = B; J.S_q = S_q; J.S_kv = S_kv; J.h = h; J.n_kv = n_kv; J.d = d;
+    J.causal = causal; J.scale = scale;
+    J.n_units = B * h;
+    return run_job(&J, n_threads);
+}
+
+/* The same, for selected query rows only: sample holds n triplets (b, i, r);
+ * out is n x d, row t being output row r of query head i in batch b. */
+int oracle_prefill_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *out,
+                        int B, int S_q, int S_kv, int h, int n_kv, int d, int causal,
+                        double scale, const int32_t *sample, int n, int n_threads) {
+    if (!check_shape(B, h, n_kv, d) || S_q <= 0 || S_kv <= 0 || n < 0) return -1;
+    for (int t = 0; t < n; ++t) {
+        const int32_t *s = sample + 3 * (size_t)t;
+        if (s[0] < 0 || s[0] >= B || s[1] < 0 || s[1] >= h || s[2] < 0 || s[2] >= S_q) return -1;
+    }
+    job_t J = {0};
+    J.kind = 0; J.q = q; J.k = k; J.v = v; J.out = out;
+    J.B = B; J.S_q = S_q; J.S_kv = S_kv; J.h = h; J.n_kv = n_kv; J.d = d;
+    J.causal = causal; J.scale = scale; J.sample = sample; J.n_sample = n;
+    J.n_units = n;
+    return run_job(&J, n_threads);
+}
+
+/* One decode step.  q [B,h,d]; caches packed [sum(max(seqlens,0)), n_kv, d]
+ * (sequence b starting at row sum of the earlier lengths); out [B,h,d] fp64.
+ * Query head i of sequence b attends to all seqlens[b] cached tokens of KV
+ * head i / (h / n_kv); a length <= 0 gives a zero row. */
+int oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                  const int32_t *seqlens, double *out, int B, int h, int n_kv, int d,
+                  double scale, int n_threads) {
+    if (!check_shape(B, h, n_kv, d)) return -1;
+    long *off = (long *)malloc(sizeof(long) * (size_t)B);
+    if (!off) return -1;
+    long acc = 0;
+    for (int b = 0; b < B; ++b) { off[b] = acc; if (seqlens[b] > 0) acc += seqlens[b]; }
+    job_t J = {0};
+    J.kind = 1; J.q = q; J.k = k_cache; J.v = v_cache; J.seqlens = seqlens; J.offsets = off;
+    J.out = out; J.B = B; J.h = h; J.n_kv = n_kv; J.d = d; J.scale = scale;
+    J.n_units = B * h;
+    int rc = run_job(&J, n_threads);
+    free(off);
+    return rc;
+}
+
+/* The softmax matrix of one prefill unit (b, i): probs is S_q x S_kv. */
+int oracle_prefill_probs(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *probs,
+                         int B, int S_q, int S_kv, int h, int n_kv, int d, int causal,
+                         double scale, int b, int i) {
+    if (!check_shape(B, h, n_kv, d) || S_q <= 0 || S_kv <= 0) return -1;
+    if (b < 0 || b >= B || i < 0 || i >= h) return -1;
+    int G = h / n_kv, g = i / G;
+    double *qd = (double *)malloc(sizeof(double) * (size_t)S_q * d);
+    double *o = (double *)malloc(sizeof(double) * (size_t)S_q * d);
+    int *vis = (int *)malloc(sizeof(int) * (size_t)S_q);
+    if (!qd || !o || !vis) { free(qd); free(o); free(vis); return -1; }
+    for (int r = 0; r < S_q; ++r) {
+        const uint16_t *qrow = q + (((size_t)b * S_q + r) * h + i) * d;
+        for (int c = 0; c < d; ++c) qd[(size_t)r * d + c] = bf16_value(qrow[c]);
+        int lim = S_kv;
+        if (causal) { int last = r + (S_kv - S_q); if (last + 1 < lim) lim = last + 1; if (lim < 0) lim = 0; }
+        vis[r] = lim;
+    }
+    int rc = attend(qd, S_q, k + ((size_t)b * S_kv * n_kv + g) * d, v + ((size_t)b * S_kv * n_kv + g) * d,
+                    (long)n_kv * d, S_kv, d, vis, scale, o, probs);
+    free(qd); free(o); free(vis);
+    return rc;
+}
