@@ -1,0 +1,14 @@
+"""B200 (sm_100a) grouped-query attention: prefill and decode through a C ABI.
+
+The work happens in ``libgqa_b200.so`` (hand-written CUDA for sm_100a, see
+``include/gqa.h``).  This package is a thin ctypes binding with the same
+names: it checks dtypes, devices and shapes, passes device pointers and the
+current CUDA stream, and raises on any non-zero status.  PyTorch is used only
+for device memory and streams.  There is no CPU fallback: if the library is
+missing, importing the binding's entry points fails loudly.
+"""
+from ._lib import (GQAError, decode, gqa_decode, gqa_get_device_status, gqa_prefill,  # noqa: F401
+                   gqa_status_string, lib, library_path, prefill)
+
+__all__ = ["prefill", "decode", "gqa_prefill", "gqa_decode", "gqa_status_string", "gqa_get_device_status",
+           "GQAError", "lib", "library_path"]

@@ -1,0 +1,148 @@
+"""ctypes binding of libgqa_b200.so: argument marshalling only."""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libgqa_b200.so")
+_lock = threading.Lock()
+_handle = None
+
+GQA_OK, GQA_ERR_INVALID_ARG, GQA_ERR_UNSUPPORTED, GQA_ERR_CUDA, GQA_ERR_TIMEOUT = range(5)
+
+# every entry point include/gqa.h declares, with its ctypes signature
+_vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+SIGNATURES = {
+    "gqa_prefill": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp], _i),
+    "gqa_decode": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
+    "gqa_status_string": ([_i], ctypes.c_char_p),
+    "gqa_get_device_status": ([_vp], _i),
+}
+
+
+class GQAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {gqa_status_string(status)} ({status})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it has not been built."""
+    global _handle
+    with _lock:
+        if _handle is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                                   "`python -m attention_gqa_decode_b200.build` (nvcc, sm_100a)")
+            h = ctypes.CDLL(_LIB_PATH)
+            for name, (args, res) in SIGNATURES.items():
+                fn = getattr(h, name)
+                fn.argtypes = args
+                fn.restype = res
+            _handle = h
+    return _handle
+
+
+def gqa_status_string(status: int) -> str:
+    return lib().gqa_status_string(int(status)).decode()
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def gqa_prefill(q, k, v, out, B, S_q, S_kv, h, n_kv, d_h, causal, scale, stream) -> int:
+    """The raw C entry point (pointers as ints); returns the status code."""
+    return lib().gqa_prefill(q, k, v, out, B, S_q, S_kv, h, n_kv, d_h, int(causal), float(scale), stream)
+
+
+def gqa_decode(q, k_cache, v_cache, seqlens, out, B, h, n_kv, d_h, scale, stream) -> int:
+    return lib().gqa_decode(q, k_cache, v_cache, seqlens, out, B, h, n_kv, d_h, float(scale), stream)
+
+
+def gqa_get_device_status(stream=None) -> int:
+    return lib().gqa_get_device_status(_stream_ptr(stream))
+
+
+def _check(t, name, ndim):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def prefill(q, k, v, causal: bool = True, scale: float | None = None, out=None, stream=None):
+    """Exact attention for q [B,S_q,h,d], k/v [B,S_kv,n_kv,d] (bf16, CUDA); returns out [B,S_q,h,d].
+
+    ``scale=None`` means 1/sqrt(d), the default of the flash_attn_func call
+    shown on the toolsku page ("Flash Attention Usage", softmax_scale=None).
+    """
+    import torch
+    _check(q, "q", 4), _check(k, "k", 4), _check(v, "v", 4)
+    B, S_q, h, d = q.shape
+    Bk, S_kv, n_kv, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk != d:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    if not (q.device == k.device == v.device):
+        raise ValueError("q, k, v must be on one device")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check(out, "out", 4)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    with torch.cuda.device(q.device):
+        st = gqa_prefill(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, S_q, S_kv, h, n_kv, d,
+                         causal, scale, _stream_ptr(stream))
+    if st != GQA_OK:
+        raise GQAError(st, "gqa_prefill")
+    return out
+
+
+def decode(q, k_cache, v_cache, seqlens, scale: float | None = None, out=None, stream=None):
+    """One decode step: q [B,h,d], packed caches [sum(seqlens),n_kv,d], seqlens int32 [B] (CUDA).
+
+    Returns out [B,h,d].  Sequence b's tokens start at cache row sum(seqlens[:b]).
+    """
+    import torch
+    _check(q, "q", 3), _check(k_cache, "k_cache", 3), _check(v_cache, "v_cache", 3)
+    B, h, d = q.shape
+    T, n_kv, dk = k_cache.shape
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or dk != d:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k_cache.shape)} v{tuple(v_cache.shape)}")
+    if not isinstance(seqlens, torch.Tensor) or seqlens.dtype != torch.int32 or not seqlens.is_cuda \
+            or seqlens.numel() != B or not seqlens.is_contiguous():
+        raise ValueError("seqlens must be a contiguous int32 CUDA tensor with B entries")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check(out, "out", 3)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    with torch.cuda.device(q.device):
+        st = gqa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(), out.data_ptr(),
+                        B, h, n_kv, d, scale, _stream_ptr(stream))
+    if st != GQA_OK:
+        raise GQAError(st, "gqa_decode")
+    return out

@@ -1,0 +1,126 @@
+// The C ABI (include/gqa.h): argument validation, dispatch, device status.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "gqa.h"
+#include "common.cuh"
+
+namespace gqa {
+__device__ int g_status = 0;   // see gqa_get_device_status()
+
+int launch_prefill(const void *q, const void *k, const void *v, void *out, int B, int S_q, int S_kv, int h, int n_kv,
+                   int d, int causal, float scale, cudaStream_t stream);
+int launch_decode(const void *q, const void *k, const void *v, const int32_t *seqlens, void *out, int B, int h,
+                  int n_kv, int d, float scale, cudaStream_t stream);
+}  // namespace gqa
+
+namespace gqa_host {
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+bool encode_tensor_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+                       const uint64_t *strides_bytes, const uint32_t *box) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[5];
+    cuuint64_t gstride[4];
+    cuuint32_t bdim[5], estride[5];
+    for (int i = 0; i < rank; ++i) {
+        gdim[i] = dims[i];
+        bdim[i] = box[i];
+        estride[i] = 1;
+        if (i + 1 < rank) gstride[i] = strides_bytes[i];
+    }
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void *>(base),
+                    gdim, gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int *device_status() {
+    static int *ptrs[64] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, gqa::g_status) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int *>(p);
+    }
+    return ptrs[dev];
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+}  // namespace gqa_host
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool scale_ok(float s) { return std::isfinite(s) && s >= 0.f; }
+
+extern "C" {
+
+int gqa_prefill(const void *q, const void *k, const void *v, void *out, int B, int S_q, int S_kv, int h, int n_kv,
+                int d_h, int causal, float scale, cudaStream_t stream) {
+    if (!q || !k || !v || !out) return GQA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GQA_ERR_INVALID_ARG;
+    if (B <= 0 || S_q <= 0 || S_kv <= 0 || h <= 0 || n_kv <= 0 || h % n_kv != 0) return GQA_ERR_INVALID_ARG;
+    if (causal && S_q > S_kv) return GQA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return GQA_ERR_INVALID_ARG;
+    if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
+    // tensor-map coordinates are int32 per dimension; the extents themselves are int already
+    return gqa::launch_prefill(q, k, v, out, B, S_q, S_kv, h, n_kv, d_h, causal, scale, stream);
+}
+
+int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens, void *out, int B,
+               int h, int n_kv, int d_h, float scale, cudaStream_t stream) {
+    if (!q || !k_cache || !v_cache || !seqlens || !out) return GQA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+        return GQA_ERR_INVALID_ARG;
+    if (B <= 0 || B > 65535 || h <= 0 || n_kv <= 0 || h % n_kv != 0) return GQA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return GQA_ERR_INVALID_ARG;
+    if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
+    if (static_cast<long>(n_kv) * ((h / n_kv + 63) / 64) > 65535) return GQA_ERR_UNSUPPORTED;
+    return gqa::launch_decode(q, k_cache, v_cache, seqlens, out, B, h, n_kv, d_h, scale, stream);
+}
+
+const char *gqa_status_string(int status) {
+    switch (status) {
+        case GQA_OK: return "GQA_OK";
+        case GQA_ERR_INVALID_ARG: return "GQA_ERR_INVALID_ARG: invalid argument";
+        case GQA_ERR_UNSUPPORTED: return "GQA_ERR_UNSUPPORTED: unsupported configuration";
+        case GQA_ERR_CUDA: return "GQA_ERR_CUDA: CUDA launch failure";
+        case GQA_ERR_TIMEOUT: return "GQA_ERR_TIMEOUT: a kernel gave up on an internal wait";
+        default: return "unknown gqa status";
+    }
+}
+
+int gqa_get_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GQA_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, gqa::g_status, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(gqa::g_status, &zero, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+    return v;
+}
+
+}  // extern "C"

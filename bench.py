@@ -1,0 +1,347 @@
+"""Benchmark: GQA decode KV GB/s (vs HBM peak) and causal prefill TFLOP/s (vs bf16 peak).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on stdout (rank 0).  A step is one decode call over the whole
+GQA decode workload (B=16 sequences, h=64, n_kv=8, d=128, 4096 cached tokens
+each), inputs resident in device memory; three copies of the KV cache are
+rotated so every step reads a cache L2 has not seen for two steps (each copy,
+256 MiB, is twice the 126 MB L2).  The causal prefill workload (B=4,
+S=4096, h=32, n_kv=8, d=128) is timed in the same run and reported under
+"prefill".  Under torchrun every rank runs the same per-GPU workload (the
+(sequence, KV head) units are independent: weak scaling, no collective on the
+data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+N_KV_COPIES = 3
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        mp = json.load(open(path))
+        return {"hbm": float(mp["hbm_gbs"]), "bf16": float(mp["bf16_tflops"]),
+                "bf16_sustained": float(mp.get("bf16_tflops_sustained", mp["bf16_tflops"])), "src": "measured"}
+    except Exception:
+        return {"hbm": FALLBACK_HBM_GBS, "bf16": FALLBACK_BF16_TFLOPS, "bf16_sustained": 1400.0, "src": "fallback"}
+
+
+def kernel_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if its source hash is current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        rec = json.load(open(path))[kernel]
+    except Exception:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return rec["bytes_per_launch"] if h == rec["source_sha256"] else None
+
+
+class ClockSampler:
+    """SM clock and throttle reasons, sampled through NVML while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4}
+
+    def __init__(self, device, period_s: float = 0.01):
+        self.device, self.period = device, period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            import torch
+            pr = torch.cuda.get_device_properties(self.device)
+            bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+            self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception:
+            self._nv = None
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------
+# CPU legs (the oracle, as it stands, on the host cores)
+
+def oracle_decode_leg(target_s: float = 10.0):
+    """Time the fp64 oracle on whole sequences of the decode workload until ~target_s."""
+    import oracle
+    import torch
+    from attention_gqa_decode_b200 import inputs, metrics
+    w = inputs.GQA_DECODE_70B
+    q, k, v, lens = inputs.workload_inputs(w)
+    per_seq = w.kv_len
+    cores = os.cpu_count() or 1
+    done_bytes, t_total, seqs = 0, 0.0, 0
+    b = 0
+    while t_total < target_s and seqs < 4 * w.B:
+        nb = min(cores, w.B)                      # one batch of sequences per call, all cores
+        b0 = (b * nb) % w.B
+        idx = [(b0 + i) % w.B for i in range(nb)]
+        qs = q[idx].contiguous()
+        ks = torch.cat([k[j * per_seq:(j + 1) * per_seq] for j in idx]).contiguous()
+        vs = torch.cat([v[j * per_seq:(j + 1) * per_seq] for j in idx]).contiguous()
+        ls = lens[idx].contiguous()
+        t0 = time.perf_counter()
+        oracle.decode(qs, ks, vs, ls, n_threads=cores)
+        t_total += time.perf_counter() - t0
+        done_bytes += metrics.decode_kv_bytes(ls.tolist(), w.n_kv, w.d)
+        seqs += nb
+        b += 1
+    return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{seqs} whole sequences of the decode workload ({w.kv_len} tokens, h={w.h}, n_kv={w.n_kv}), "
+                      f"{t_total:.1f} s of fp64 oracle time"}
+
+
+# ----------------------------------------------------------------------------
+# GPU legs
+
+def time_launches(fn, steps, warmup, stream, flush=None):
+    """CUDA-event time of each launch of fn(step) on `stream`; returns per-step ms list and total ms."""
+    import torch
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    tot0, tot1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tot0.record(stream)
+    for i in range(steps):
+        if flush is not None:
+            flush(i)
+        ev[i][0].record(stream)
+        fn(i)
+        ev[i][1].record(stream)
+    tot1.record(stream)
+    torch.cuda.synchronize()
+    per = [a.elapsed_time(b) for a, b in ev]
+    return per, tot0.elapsed_time(tot1)
+
+
+def decode_leg(args, device, world, clocks):
+    import torch
+    import attention_gqa_decode_b200 as gqa
+    from attention_gqa_decode_b200 import inputs, metrics
+    w = inputs.GQA_DECODE_70B
+    q, k, v, lens = inputs.workload_inputs(w)
+    kv_bytes = metrics.decode_kv_bytes(lens.tolist(), w.n_kv, w.d)
+    qd, ld = q.to(device), lens.to(device)
+    ks = [k.to(device) for _ in range(N_KV_COPIES)]
+    vs = [v.to(device) for _ in range(N_KV_COPIES)]
+    out = torch.empty_like(qd)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i):
+        c = i % N_KV_COPIES
+        gqa.decode(qd, ks[c], vs[c], ld, out=out)
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with clocks:
+        per, total = time_launches(step, args.steps, args.warmup, stream)
+    barrier(world)
+    total_max = max_over_ranks(total, world, device)
+    kern_ms = statistics.mean(per)
+    st = gqa.gqa_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the decode leg")
+    res = {"kv_bytes": kv_bytes, "total_ms": total_max, "kernel_ms": kern_ms, "per_ms": per}
+
+    # end to end through the public API: pinned host inputs -> device -> decode -> host result
+    qh, kh, vh, lh = (t.pin_memory() for t in (q, k, v, lens))
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    qe, ke, ve, le = (torch.empty_like(t, device=device) for t in (q, k, v, lens))
+    e2e_steps = max(3, min(10, args.steps))
+
+    def e2e(i):
+        qe.copy_(qh, non_blocking=True)
+        ke.copy_(kh, non_blocking=True)
+        ve.copy_(vh, non_blocking=True)
+        le.copy_(lh, non_blocking=True)
+        o = gqa.decode(qe, ke, ve, le)
+        oh.copy_(o, non_blocking=True)
+
+    barrier(world)
+    per_e, total_e = time_launches(e2e, e2e_steps, 2, stream)
+    barrier(world)
+    total_e = max_over_ranks(total_e, world, device)
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v, lens))
+    d2h = oh.numel() * oh.element_size()
+    res["e2e"] = {"value": world * kv_bytes * e2e_steps / (total_e / 1e3) / 1e9, "unit": "GB/s",
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    return res
+
+
+def prefill_leg(args, device, world):
+    import torch
+    import attention_gqa_decode_b200 as gqa
+    from attention_gqa_decode_b200 import inputs, metrics
+    w = inputs.GQA_CAUSAL_PREFILL
+    q, k, v = inputs.workload_inputs(w)
+    flops = metrics.prefill_flops(w.B, w.S_q, w.S_kv, w.h, w.d, True)
+    qd, kd, vd = q.to(device), k.to(device), v.to(device)
+    out = torch.empty_like(qd)
+    stream = torch.cuda.current_stream(device)
+    scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)   # > L2: flushed between steps
+
+    def flush(i):
+        scratch.fill_(i & 0xFF)
+
+    steps = max(3, min(args.steps, 30))
+    barrier(world)
+    per, _ = time_launches(lambda i: gqa.prefill(qd, kd, vd, causal=True, out=out), steps, max(3, args.warmup),
+                           stream, flush=flush)
+    barrier(world)
+    kern_ms = max_over_ranks(statistics.mean(per), world, device)
+    if gqa.gqa_get_device_status() != 0:
+        raise RuntimeError("device status after the prefill leg")
+    return {"flops": flops, "kernel_ms": kern_ms, "steps": steps,
+            "io_bytes": metrics.prefill_io_bytes(w.B, w.S_q, w.S_kv, w.h, w.n_kv, w.d)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank, world, local = dist_env()
+    from attention_gqa_decode_b200 import inputs
+    w = inputs.GQA_DECODE_70B
+    metric = "GQA decode KV GB/s"
+    config = {"workload": w.name, "B": w.B, "h": w.h, "n_kv": w.n_kv, "d_h": w.d, "kv_len": w.kv_len,
+              "global_batch": w.B * world, "parallelism": f"dp{world}" if world > 1 else "single",
+              "l2": f"{N_KV_COPIES} KV copies of 256 MiB rotated (each step reads a cache unseen for 2 steps)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cpu = oracle_decode_leg(target_s=min(60.0, 5.0 + 0.2 * args.steps))
+        line = {"impl": "reference", "metric": metric, "value": cpu["value"], "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16 inputs)",
+                "config": config, "cpu_baseline": cpu,
+                "e2e": {"value": cpu["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    pk = peaks()
+    clocks = ClockSampler(device)
+    dec = decode_leg(args, device, world, clocks)
+    pre = None if args.no_prefill else prefill_leg(args, device, world)
+
+    value = world * dec["kv_bytes"] * args.steps / (dec["total_ms"] / 1e3) / 1e9
+    achieved = dec["kv_bytes"] / (dec["kernel_ms"] / 1e3) / 1e9
+    line = {
+        "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dec["total_ms"] / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v)", "config": config,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm"], "traffic": kernel_traffic("gqa_decode_kernel"),
+                     "algorithmic_bytes_per_launch": dec["kv_bytes"], "peak_source": pk["src"]},
+        "e2e": dec["e2e"],
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    if pre is not None:
+        tf = pre["flops"] / (pre["kernel_ms"] / 1e3) / 1e12
+        line["prefill"] = {
+            "metric": "GQA causal prefill TFLOP/s", "workload": inputs.GQA_CAUSAL_PREFILL.name,
+            "value": world * tf, "unit": "TFLOP/s", "ms_per_call": pre["kernel_ms"], "steps": pre["steps"],
+            "l2": "256 MiB buffer written between calls",
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16"], "unit": "TFLOP/s",
+                         "frac": tf / pk["bf16"], "frac_of_sustained": tf / pk["bf16_sustained"],
+                         "traffic": kernel_traffic("gqa_prefill_kernel"),
+                         "algorithmic_flops_per_launch": pre["flops"], "peak_source": pk["src"]}}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_decode_leg(target_s=10.0)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

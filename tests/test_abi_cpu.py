@@ -1,0 +1,89 @@
+"""The C-ABI library without a GPU: it loads, exports every declared entry
+point, and rejects invalid arguments synchronously (nothing is launched on
+these paths, so no device is needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import attention_gqa_decode_b200 as gqa
+from attention_gqa_decode_b200 import _lib
+from attention_gqa_decode_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return gqa.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "gqa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(gqa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    assert declared_functions() == sorted(_lib.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert isinstance(getattr(L, name), ctypes._CFuncPtr), name
+
+
+def test_status_strings(L):
+    for code in range(5):
+        assert gqa.gqa_status_string(code).startswith("GQA_")
+    assert "unknown" in gqa.gqa_status_string(99)
+
+
+A = 1 << 20        # a 16-byte-aligned fake address; never dereferenced on these paths
+BAD = A + 2        # misaligned
+
+
+@pytest.mark.parametrize("args,expect", [
+    # q, k, v, out, B, S_q, S_kv, h, n_kv, d, causal, scale
+    ((0, A, A, A, 1, 8, 8, 4, 1, 64, 1, 0.125), _lib.GQA_ERR_INVALID_ARG),     # null pointer
+    ((A, BAD, A, A, 1, 8, 8, 4, 1, 64, 1, 0.125), _lib.GQA_ERR_INVALID_ARG),   # misaligned
+    ((A, A, A, A, 0, 8, 8, 4, 1, 64, 1, 0.125), _lib.GQA_ERR_INVALID_ARG),     # B = 0
+    ((A, A, A, A, 1, 0, 8, 4, 1, 64, 1, 0.125), _lib.GQA_ERR_INVALID_ARG),     # S_q = 0
+    ((A, A, A, A, 1, 8, -1, 4, 1, 64, 1, 0.125), _lib.GQA_ERR_INVALID_ARG),    # S_kv < 0
+    ((A, A, A, A, 1, 8, 8, 6, 4, 64, 1, 0.125), _lib.GQA_ERR_INVALID_ARG),     # h % n_kv != 0
+    ((A, A, A, A, 1, 9, 8, 4, 1, 64, 1, 0.125), _lib.GQA_ERR_INVALID_ARG),     # causal, S_q > S_kv
+    ((A, A, A, A, 1, 8, 8, 4, 1, 64, 1, float("nan")), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, 1, 8, 8, 4, 1, 64, 1, float("inf")), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, 1, 8, 8, 4, 1, 64, 1, -0.5), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, 1, 8, 8, 4, 1, 96, 1, 0.125), _lib.GQA_ERR_UNSUPPORTED),     # d_h = 96
+    ((A, A, A, A, 1, 8, 8, 4, 1, 256, 0, 0.125), _lib.GQA_ERR_UNSUPPORTED),
+])
+def test_prefill_rejects(L, args, expect):
+    assert gqa.gqa_prefill(*args, None) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    # q, k, v, seqlens, out, B, h, n_kv, d, scale
+    ((A, A, A, 0, A, 2, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),       # null seqlens
+    ((A, A, A, A + 1, A, 2, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),   # misaligned seqlens
+    ((A, A, BAD, A, A, 2, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, A, 0, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, A, 65536, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),   # B above the grid limit
+    ((A, A, A, A, A, 2, 4, 3, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, A, 2, 0, 1, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, A, 2, 4, 2, 128, float("nan")), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, A, 2, 4, 2, 32, 0.1), _lib.GQA_ERR_UNSUPPORTED),
+])
+def test_decode_rejects(L, args, expect):
+    assert gqa.gqa_decode(*args, None) == expect
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        gqa.prefill(q, q[:, :, :1].contiguous(), q[:, :, :1].contiguous())
+    with pytest.raises(TypeError):
+        gqa.prefill(q.float(), q, q)

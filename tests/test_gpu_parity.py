@@ -1,0 +1,203 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerance (fixed for this method: bf16 inputs and outputs, fp32 accumulation):
+max |GPU - oracle| <= 1e-2 and mean |GPU - oracle| <= 1e-3 per call, the
+oracle being unrounded fp64.  Index and group-mapping work is checked
+bit-exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import attention_gqa_decode_b200 as gqa
+import oracle
+from attention_gqa_decode_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 1e-2
+MEAN_ABS = 1e-3
+
+
+def dev(*ts):
+    return [t.cuda() for t in ts]
+
+
+def check(got: torch.Tensor, ref: np.ndarray, what: str):
+    g = got.detach().float().cpu().double().numpy()
+    assert g.shape == ref.shape, (g.shape, ref.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    err = np.abs(g - ref)
+    mx, mean = float(err.max()), float(err.mean())
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max abs {mx:.3e}, mean abs {mean:.3e}"
+    return mx, mean
+
+
+def gpu_decode(q, k, v, lens, scale=None):
+    qd, kd, vd, ld = dev(q, k, v, lens)
+    out = gqa.decode(qd, kd, vd, ld, scale=scale)
+    torch.cuda.synchronize()
+    return out.cpu()
+
+
+def gpu_prefill(q, k, v, causal=True, scale=None):
+    qd, kd, vd = dev(q, k, v)
+    out = gqa.prefill(qd, kd, vd, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    return out.cpu()
+
+
+# ----------------------------------------------------------------------------
+# the named workloads
+
+@pytest.mark.parametrize("w", [inputs.GQA_DECODE_70B, inputs.MQA_DECODE_LONG] + list(inputs.RAGGED_SWEEP),
+                         ids=lambda w: w.name)
+def test_decode_workload(w):
+    q, k, v, lens = inputs.workload_inputs(w)
+    check(gpu_decode(q, k, v, lens), oracle.decode(q, k, v, lens), w.name)
+
+
+def test_prefill_tiny_mqa():
+    w = inputs.TINY_MQA_PREFILL
+    q, k, v = inputs.workload_inputs(w)
+    got = gpu_prefill(q, k, v, causal=True)
+    check(got, oracle.prefill(q, k, v, causal=True), w.name)
+    # row 0 attends to key 0 alone: exactly V[0] of its group
+    for i in range(w.h):
+        assert torch.equal(got[0, 0, i], v[0, 0, i // w.G]), i
+
+
+def test_prefill_gqa_causal_sampled():
+    """The full-size causal prefill, in the launch configuration the bench times,
+    checked on sampled rows the oracle computes one by one."""
+    w = inputs.GQA_CAUSAL_PREFILL
+    q, k, v = inputs.workload_inputs(w)
+    got = gpu_prefill(q, k, v, causal=True)
+    rng = np.random.default_rng(4)
+    rows = [0, 1, 127, 128, 129, 255, 256, 511, 2047, 2048, 4095] + list(rng.integers(0, w.S_q, 40))
+    sample = [(int(rng.integers(0, w.B)), int(rng.integers(0, w.h)), int(r)) for r in rows]
+    sample += [(w.B - 1, w.h - 1, w.S_q - 1), (0, 0, w.S_q - 1)]
+    ref = oracle.prefill_rows(q, k, v, sample, causal=True)
+    g = torch.stack([got[b, r, i] for b, i, r in sample])
+    check(g, ref, w.name)
+    assert torch.isfinite(got.float()).all()
+
+
+# ----------------------------------------------------------------------------
+# shapes: ragged tails, several tiles, bottom-right causal, d 64/128, the spectrum
+
+@pytest.mark.parametrize("B,S_q,S_kv,h,n_kv,d,causal", [
+    (1, 300, 300, 4, 2, 128, True),     # ragged tail over 3 key tiles
+    (2, 200, 200, 6, 3, 64, False),
+    (1, 100, 333, 8, 8, 128, True),     # MHA, bottom-right causal, S_q < S_kv
+    (1, 257, 513, 4, 1, 64, True),      # MQA
+    (1, 1, 1, 2, 1, 128, True),         # one query, one key
+    (2, 129, 129, 3, 1, 128, True),
+    (1, 384, 384, 2, 2, 64, False),
+    (1, 640, 640, 2, 1, 128, True),     # several query-tile pairs
+    (1, 64, 1000, 4, 2, 128, False),
+])
+def test_prefill_shapes(B, S_q, S_kv, h, n_kv, d, causal):
+    q, k, v = inputs.prefill_inputs(100 + S_q, B, S_q, S_kv, h, n_kv, d)
+    check(gpu_prefill(q, k, v, causal=causal), oracle.prefill(q, k, v, causal=causal), "prefill")
+
+
+@pytest.mark.parametrize("G", [1, 3, 8, 12, 16, 24, 32, 48, 64, 128])
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_group_sizes(G, d):
+    n_kv = 2
+    lens = torch.tensor([0, 1, 63, 64, 65, 130, 1000, 17], dtype=torch.int32)
+    q, k, v, lens = inputs.decode_inputs(G * 7 + d, len(lens), G * n_kv, n_kv, d, lens)
+    got = gpu_decode(q, k, v, lens)
+    check(got, oracle.decode(q, k, v, lens), f"decode G={G} d={d}")
+    assert torch.all(got[0] == 0)           # zero-length sequence -> zero row
+
+
+# ----------------------------------------------------------------------------
+# properties with exact answers
+
+def test_single_key_is_exact():
+    lens = torch.ones(5, dtype=torch.int32)
+    q, k, v, lens = inputs.decode_inputs(3, 5, 16, 4, 128, lens)
+    got = gpu_decode(q, k, v, lens)
+    for b in range(5):
+        for i in range(16):
+            assert torch.equal(got[b, i], v[b, i // 4]), (b, i)
+
+
+def test_group_mapping_bit_exact():
+    h, n_kv, d = 32, 8, 128
+    q, k, v, lens = inputs.decode_inputs(5, 3, h, n_kv, d, 300)
+    vg = torch.arange(n_kv, dtype=torch.float32).view(1, n_kv, 1).expand(v.shape[0], n_kv, d).to(torch.bfloat16)
+    got = gpu_decode(q, k, vg.contiguous(), lens)
+    want = torch.arange(h).div(h // n_kv, rounding_mode="floor").float().view(1, h, 1).expand(3, h, d)
+    assert torch.equal(got.float(), want)
+    qp, kp, vp = inputs.prefill_inputs(5, 1, 200, 200, h, n_kv, d)
+    vg = torch.arange(n_kv, dtype=torch.float32).view(1, 1, n_kv, 1).expand(1, 200, n_kv, d).to(torch.bfloat16)
+    got = gpu_prefill(qp, kp, vg.contiguous(), causal=True)
+    want = torch.arange(h).div(h // n_kv, rounding_mode="floor").float().view(1, 1, h, 1).expand(1, 200, h, d)
+    assert torch.equal(got.float(), want)
+
+
+def test_zero_scale_is_mean_of_v():
+    q, k, v, lens = inputs.decode_inputs(8, 2, 8, 2, 128, torch.tensor([700, 5], dtype=torch.int32))
+    check(gpu_decode(q, k, v, lens, scale=0.0), oracle.decode(q, k, v, lens, scale=0.0), "scale 0 decode")
+    q, k, v = inputs.prefill_inputs(8, 1, 150, 150, 4, 2, 64)
+    check(gpu_prefill(q, k, v, scale=0.0), oracle.prefill(q, k, v, scale=0.0), "scale 0 prefill")
+
+
+def test_large_scores_stay_finite():
+    """Scores far from 0 exercise the running-max rescaling."""
+    q, k, v = inputs.prefill_inputs(9, 1, 300, 300, 2, 1, 128)
+    q = (q.float() * 4).to(torch.bfloat16)
+    check(gpu_prefill(q, k, v, causal=True), oracle.prefill(q, k, v, causal=True), "large scores prefill")
+    q2, k2, v2, lens = inputs.decode_inputs(9, 2, 8, 1, 128, 900)
+    q2 = (q2.float() * 4).to(torch.bfloat16)
+    check(gpu_decode(q2, k2, v2, lens), oracle.decode(q2, k2, v2, lens), "large scores decode")
+
+
+def test_split_count_does_not_change_the_result():
+    """One sequence alone (many splits per sequence) and inside a large batch (few)."""
+    h, n_kv, d, L = 16, 2, 128, 3000
+    q, k, v, lens = inputs.decode_inputs(12, 1, h, n_kv, d, L)
+    alone = gpu_decode(q, k, v, lens)
+    Bb = 200
+    qb = q.expand(Bb, h, d).contiguous()
+    kb = k.repeat(Bb, 1, 1)
+    vb = v.repeat(Bb, 1, 1)
+    batch = gpu_decode(qb, kb, vb, torch.full((Bb,), L, dtype=torch.int32))
+    diff = (batch.float() - alone.float()).abs().max().item()
+    assert diff <= 4e-3, diff
+    assert torch.equal(batch[0], batch[-1])
+
+
+def test_gqa_equals_mha_on_repeated_kv():
+    h, n_kv, d = 16, 4, 128
+    q, k, v, lens = inputs.decode_inputs(13, 3, h, n_kv, d, torch.tensor([100, 2000, 777], dtype=torch.int32))
+    rep = lambda t: t.repeat_interleave(h // n_kv, dim=1).contiguous()
+    a = gpu_decode(q, k, v, lens)
+    b = gpu_decode(q, rep(k), rep(v), lens)
+    assert (a.float() - b.float()).abs().max().item() <= 4e-3
+
+
+def test_prefill_last_row_matches_decode():
+    B, S, h, n_kv, d = 2, 333, 8, 2, 128
+    q, k, v = inputs.prefill_inputs(14, B, S, S, h, n_kv, d)
+    pre = gpu_prefill(q, k, v, causal=True)
+    dec = gpu_decode(q[:, -1].contiguous(), k.reshape(B * S, n_kv, d), v.reshape(B * S, n_kv, d),
+                     torch.full((B,), S, dtype=torch.int32))
+    assert (pre[:, -1].float() - dec.float()).abs().max().item() <= 1e-2
+
+
+def test_repeatable():
+    q, k, v, lens = inputs.workload_inputs(inputs.GQA_DECODE_70B)
+    qd, kd, vd, ld = dev(q, k, v, lens)
+    a = gqa.decode(qd, kd, vd, ld)
+    b = gqa.decode(qd, kd, vd, ld)
+    assert torch.equal(a, b)
+    qp, kp, vp = dev(*inputs.prefill_inputs(1, 1, 512, 512, 8, 2, 128))
+    assert torch.equal(gqa.prefill(qp, kp, vp), gqa.prefill(qp, kp, vp))
+
+
+def test_device_status_clean():
+    assert gqa.gqa_get_device_status() == 0
