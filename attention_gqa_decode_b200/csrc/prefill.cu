@@ -235,20 +235,31 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const bool landed = mbar_wait(&sfull[t], j & 1, abort_flag, p.status);
             if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }   // tcgen05.ld/st are warp-aligned
             tc_fence_after();
-            // pass 1: the row maximum (S stays in TMEM; reading it twice keeps
-            // the register footprint within the 168 a 10-warp CTA allows)
+            // pass 1: the row maximum (S stays in TMEM and is read again in pass
+            // 2: the 168 registers a 10-warp CTA allows cannot hold S and P)
             const int key0 = j * kPfKeys;
             const bool masked = key0 + kPfKeys - 1 > limit;
-            float mx = -INFINITY;
+            float mx;
+            {
+                uint32_t raw[4][32];
 #pragma unroll
-            for (int ch = 0; ch < kPfKeys / 32; ++ch) {
-                uint32_t raw[32];
-                tmem_ld32(tS + ch * 32, raw);
+                for (int ch = 0; ch < 4; ++ch) tmem_ld32(tS + ch * 32, raw[ch]);
                 tmem_wait_ld();
+                if (!masked) {
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float v = __uint_as_float(raw[e]);
-                    mx = (masked && key0 + ch * 32 + e > limit) ? mx : fmaxf(mx, v);
+                    for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2)
+                            m4[ch] = fmax3(m4[ch], __uint_as_float(raw[ch][e]), __uint_as_float(raw[ch][e + 1]));
+                    mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                } else {
+                    mx = -INFINITY;
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (key0 + ch * 32 + e <= limit) mx = fmaxf(mx, __uint_as_float(raw[ch][e]));
                 }
             }
             const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * cl2;
@@ -273,28 +284,37 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     m_used = m_new;
                 }
             }
-            // pass 2: P = exp2(S * scale * log2(e) - m), packed bf16, written back over S
-            float rs = 0.f;
-#pragma unroll
-            for (int ch = 0; ch < kPfKeys / 32; ++ch) {
-                uint32_t raw[32];
-                tmem_ld32(tS + ch * 32, raw);
+            // pass 2: P = exp2(S * scale * log2(e) - m), packed bf16, written back
+            // over S; the next chunk's TMEM load is in flight while this one is
+            // computed.  The running sum adds the rounded weights.
+            float2 rs2 = make_float2(0.f, 0.f);
+            {
+                uint32_t raw[2][32];
+                tmem_ld32(tS, raw[0]);
                 tmem_wait_ld();
-                uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int c = ch * 32 + 2 * e;
-                    float a = exp2f(fmaf(__uint_as_float(raw[2 * e]), cl2, -m_used));
-                    float bb = exp2f(fmaf(__uint_as_float(raw[2 * e + 1]), cl2, -m_used));
-                    if (masked) {
-                        a = (key0 + c > limit) ? 0.f : a;
-                        bb = (key0 + c + 1 > limit) ? 0.f : bb;
+                for (int ch = 0; ch < 4; ++ch) {
+                    if (ch + 1 < 4) tmem_ld32(tS + (ch + 1) * 32, raw[(ch + 1) & 1]);
+                    const uint32_t(&r)[32] = raw[ch & 1];
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float2 x = ffma2_bcast(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), cl2,
+                                                     -m_used);
+                        float a = exp2f(x.x), bb = exp2f(x.y);
+                        if (masked) {
+                            const int c = ch * 32 + 2 * e;
+                            a = (key0 + c > limit) ? 0.f : a;
+                            bb = (key0 + c + 1 > limit) ? 0.f : bb;
+                        }
+                        pk[e] = pack_bf16x2(a, bb);
+                        rs2 = fadd2(rs2, unpack_bf16x2(pk[e]));
                     }
-                    pk[e] = pack_bf16x2(a, bb);
-                    rs += sum_bf16x2(pk[e]);
+                    tmem_st16(tS + ch * 16, pk);
+                    if (ch + 1 < 4) tmem_wait_ld();
                 }
-                tmem_st16(tS + ch * 16, pk);
             }
+            const float rs = rs2.x + rs2.y;
             l += rs;
             tmem_wait_st();
             tc_fence_before();
