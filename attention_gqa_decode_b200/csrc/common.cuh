@@ -339,4 +339,5 @@ int sm_count();
 // Device address of the library's status word on the current device (null on failure).
 int *device_status();
 
+
 }  // namespace gqa_host

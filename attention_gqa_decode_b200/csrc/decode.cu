@@ -25,7 +25,16 @@
 //     scratch memory is used.
 #include <cooperative_groups.h>
 
+#include <algorithm>
+
 #include "common.cuh"
+
+#ifndef GQA_DECODE_CTAS_PER_SM
+#define GQA_DECODE_CTAS_PER_SM 2   // resident CTAs per SM (shared memory allows two)
+#endif
+#ifndef GQA_DECODE_MAX_SPLIT
+#define GQA_DECODE_MAX_SPLIT 8     // splits per (sequence, KV head) = thread-block cluster size
+#endif
 
 namespace cg = cooperative_groups;
 
@@ -222,8 +231,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
             for (int nt = 0; nt < NTS; ++nt) {
-                mx[0] = fmaxf(mx[0], fmaxf(s[nt][0], s[nt][1]));
-                mx[1] = fmaxf(mx[1], fmaxf(s[nt][2], s[nt][3]));
+                mx[0] = fmax3(mx[0], s[nt][0], s[nt][1]);
+                mx[1] = fmax3(mx[1], s[nt][2], s[nt][3]);
             }
             float alpha[2];
 #pragma unroll
@@ -242,31 +251,33 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                 o[nt][2] *= alpha[1];
                 o[nt][3] *= alpha[1];
             }
+            // P as bf16 A fragments; the running sums add the rounded weights
+            uint32_t pa[KKS][4];
+            float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int nt = 0; nt < NTS; ++nt) {
-                s[nt][0] = exp2f(fmaf(s[nt][0], cl2, -m_run[0]));
-                s[nt][1] = exp2f(fmaf(s[nt][1], cl2, -m_run[0]));
-                s[nt][2] = exp2f(fmaf(s[nt][2], cl2, -m_run[1]));
-                s[nt][3] = exp2f(fmaf(s[nt][3], cl2, -m_run[1]));
+                const float2 x0 = ffma2_bcast(s[nt][0], s[nt][1], cl2, -m_run[0]);
+                const float2 x1 = ffma2_bcast(s[nt][2], s[nt][3], cl2, -m_run[1]);
+                float e0 = exp2f(x0.x), e1 = exp2f(x0.y), e2 = exp2f(x1.x), e3 = exp2f(x1.y);
+                if (partial) {   // masked tokens add nothing (also when scale == 0)
+                    const int tok = tw0 + nt * 8 + cq;
+                    if (tok < row_lo) {
+                        e0 = 0.f;
+                        e2 = 0.f;
+                    }
+                    if (tok + 1 < row_lo) {
+                        e1 = 0.f;
+                        e3 = 0.f;
+                    }
+                }
+                const uint32_t lo = pack_bf16x2(e0, e1), hi = pack_bf16x2(e2, e3);
+                pa[nt >> 1][(nt & 1) * 2 + 0] = lo;
+                pa[nt >> 1][(nt & 1) * 2 + 1] = hi;
+                ls0 = fadd2(ls0, unpack_bf16x2(lo));
+                ls1 = fadd2(ls1, unpack_bf16x2(hi));
             }
-            if (partial) {   // masked tokens contribute nothing (also when scale == 0)
-#pragma unroll
-                for (int nt = 0; nt < NTS; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        if (tw0 + nt * 8 + cq + (e & 1) < row_lo) s[nt][e] = 0.f;
-            }
-            // P as bf16 A fragments; the running sum adds the rounded weights
-            uint32_t pa[KKS][4];
-#pragma unroll
-            for (int kk = 0; kk < KKS; ++kk) {
-                pa[kk][0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
-                pa[kk][1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
-                pa[kk][2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-                pa[kk][3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-                l_run[0] += sum_bf16x2(pa[kk][0]) + sum_bf16x2(pa[kk][2]);
-                l_run[1] += sum_bf16x2(pa[kk][1]) + sum_bf16x2(pa[kk][3]);
-            }
+            l_run[0] += ls0.x + ls0.y;
+            l_run[1] += ls1.x + ls1.y;
             // O += P V
 #pragma unroll
             for (int kk = 0; kk < KKS; ++kk) {
@@ -382,6 +393,9 @@ static int launch_decode_t(const void *q, const void *k, const void *v, const in
     if (dev < 64 && !(attr_done >> dev & 1ull)) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal) != cudaSuccess)
             return 3;
+        if (GQA_DECODE_MAX_SPLIT > 8 &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+            return 3;
         attr_done |= 1ull << dev;
     }
     CUtensorMap tk, tv;
@@ -395,8 +409,11 @@ static int launch_decode_t(const void *q, const void *k, const void *v, const in
     const int slices = (G + kDecMaxHeads - 1) / kDecMaxHeads;
     const long units = static_cast<long>(B) * n_kv * slices;
     const int sms = gqa_host::sm_count();
-    int P = 1;   // splits per (b, g): enough CTAs to cover every SM twice, at most 8 (portable cluster)
-    while (P < 8 && units * P < 2L * sms) P *= 2;
+    // Splits per (sequence, KV head): as many as fit in one wave of resident
+    // CTAs (two per SM), at most the cluster limit.  Longer CTAs amortise their
+    // start and merge; a second, partial wave would leave SMs idle at the end.
+    const long slots = static_cast<long>(GQA_DECODE_CTAS_PER_SM) * sms;
+    const int P = static_cast<int>(std::max(1L, std::min(static_cast<long>(GQA_DECODE_MAX_SPLIT), slots / units)));
 
     DecodeParams prm;
     prm.q = static_cast<const __nv_bfloat16 *>(q);
