@@ -26,6 +26,8 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from attention_gqa_decode_b200 import multirank  # noqa: E402
+
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 N_KV_COPIES = 3
@@ -109,16 +111,6 @@ class ClockSampler:
 
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
-
-
-def max_over_ranks(x: float, world: int, device) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
 
 
 def barrier(world):
@@ -206,7 +198,7 @@ def decode_leg(args, device, world, clocks):
     with clocks:
         per, total = time_launches(step, args.steps, args.warmup, stream)
     barrier(world)
-    total_max = max_over_ranks(total, world, device)
+    total_max = multirank.max_over_ranks(total, device)
     kern_ms = statistics.mean(per)
     st = gqa.gqa_get_device_status()
     if st != 0:
@@ -230,10 +222,10 @@ def decode_leg(args, device, world, clocks):
     barrier(world)
     per_e, total_e = time_launches(e2e, e2e_steps, 2, stream)
     barrier(world)
-    total_e = max_over_ranks(total_e, world, device)
+    total_e = multirank.max_over_ranks(total_e, device)
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v, lens))
     d2h = oh.numel() * oh.element_size()
-    res["e2e"] = {"value": world * kv_bytes * e2e_steps / (total_e / 1e3) / 1e9, "unit": "GB/s",
+    res["e2e"] = {"value": multirank.job_throughput(kv_bytes * e2e_steps, total_e, device) / 1e9, "unit": "GB/s",
                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     return res
 
@@ -258,7 +250,7 @@ def prefill_leg(args, device, world):
     per, _ = time_launches(lambda i: gqa.prefill(qd, kd, vd, causal=True, out=out), steps, max(3, args.warmup),
                            stream, flush=flush)
     barrier(world)
-    kern_ms = max_over_ranks(statistics.mean(per), world, device)
+    kern_ms = multirank.max_over_ranks(statistics.mean(per), device)
     if gqa.gqa_get_device_status() != 0:
         raise RuntimeError("device status after the prefill leg")
     return {"flops": flops, "kernel_ms": kern_ms, "steps": steps,
@@ -308,7 +300,7 @@ def main():
     dec = decode_leg(args, device, world, clocks)
     pre = None if args.no_prefill else prefill_leg(args, device, world)
 
-    value = world * dec["kv_bytes"] * args.steps / (dec["total_ms"] / 1e3) / 1e9
+    value = multirank.job_throughput(dec["kv_bytes"] * args.steps, dec["total_ms"], device) / 1e9
     achieved = dec["kv_bytes"] / (dec["kernel_ms"] / 1e3) / 1e9
     line = {
         "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
