@@ -295,6 +295,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
+// Move registers between warpgroups (every warp of the warpgroup executes it).
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand (sm_100
 // format): start address >> 4 in bits 0-13, leading-dimension byte offset
 // >> 4 in bits 16-29, stride-dimension byte offset >> 4 in bits 32-45,

@@ -18,11 +18,12 @@
 //               TMEM, and O_t += P_t V (A = P_t read from TMEM, B = V
 //               MN-major from shared memory), committing to mbarriers;
 //   warps 0-7   two softmax warpgroups, one per query tile (thread = query
-//               row = TMEM lane): load the S row, mask (causal diagonal and
-//               ragged tail), running max with lazy rescaling of O in TMEM
-//               (only when the max grows by more than 2^8), exp2 with the
-//               scale folded in, P as packed bf16 written back over S, then
-//               the epilogue O / l -> bf16 -> global.
+//               row = TMEM lane), holding 216 registers each (setmaxnreg;
+//               warps 8-11 give theirs up): load the whole S row from TMEM
+//               once, mask (causal diagonal and ragged tail), running max
+//               with lazy rescaling of O in TMEM (only when the max grows by
+//               more than 2^8), exp2 with the scale folded in, P as packed
+//               bf16 written back over S, then the epilogue O / l -> bf16.
 // The two query tiles ping-pong: while one warpgroup computes its softmax,
 // the tensor cores run the other tile's P V and next Q K^T.  Causal CTAs are
 // ordered heaviest first; tiles wholly above the diagonal are never loaded.
@@ -33,7 +34,12 @@ namespace gqa {
 constexpr int kPfRows = 128;     // query rows per tile (MMA M)
 constexpr int kPfKeys = 128;     // keys per KV tile
 constexpr int kPfRing = 5;       // K/V tiles in flight
-constexpr int kPfThreads = 320;  // 8 softmax warps + producer + MMA
+constexpr int kPfThreads = 384;  // softmax warpgroups 0 and 1; warpgroup 2 = producer, MMA, 2 idle warps
+// Register split (setmaxnreg): the launch gives 168 per thread (384 x 168 =
+// 64512); warpgroup 2 drops to 64 and the softmax warpgroups rise to 216:
+// 256 x 216 + 128 x 64 = 63488 <= 64512.
+constexpr uint32_t kRegsSoftmax = 216, kRegsOther = 64;
+static_assert(256 * kRegsSoftmax + 128 * kRegsOther <= kPfThreads * 168, "register split exceeds the launch");
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 struct PrefillParams {
@@ -117,107 +123,111 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-            mbar_arrive_expect_tx(qfull, SM::kQ);
-            for (int t = 0; t < 2; ++t)
-                for (int hf = 0; hf < D / 64; ++hf)
-                    tma_load_4d(sQ + t * SM::kTile + hf * SM::kHalf, &tm_q, qfull, hf * 64, head, q0 + t * kPfRows, b);
-            int item = 0;
-            bool stop = false;
-            for (int j = 0; j < nmax && !stop; ++j) {
-                for (int kv = 0; kv < 2; ++kv, ++item) {
-                    const int slot = item % kPfRing, use = item / kPfRing;
-                    if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, abort_flag, p.status)) { stop = true; break; }
-                    mbar_arrive_expect_tx(&full[slot], SM::kTile);
-                    const CUtensorMap *map = kv ? &tm_v : &tm_k;
+    if (warp >= 8) {
+        regs_dec<kRegsOther>();   // warpgroup 2: producer, MMA issuer, two idle warps
+        if (warp == 8) {
+            // ------------------------------------------------------------ producer
+            if (lane == 0) {
+                tma_prefetch_desc(&tm_q);
+                tma_prefetch_desc(&tm_k);
+                tma_prefetch_desc(&tm_v);
+                mbar_arrive_expect_tx(qfull, SM::kQ);
+                for (int t = 0; t < 2; ++t)
                     for (int hf = 0; hf < D / 64; ++hf)
-                        tma_load_4d(sRing + slot * SM::kTile + hf * SM::kHalf, map, &full[slot], hf * 64, kvh,
-                                    j * kPfKeys, b);
+                        tma_load_4d(sQ + t * SM::kTile + hf * SM::kHalf, &tm_q, qfull, hf * 64, head, q0 + t * kPfRows, b);
+                int item = 0;
+                bool stop = false;
+                for (int j = 0; j < nmax && !stop; ++j) {
+                    for (int kv = 0; kv < 2; ++kv, ++item) {
+                        const int slot = item % kPfRing, use = item / kPfRing;
+                        if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, abort_flag, p.status)) { stop = true; break; }
+                        mbar_arrive_expect_tx(&full[slot], SM::kTile);
+                        const CUtensorMap *map = kv ? &tm_v : &tm_k;
+                        for (int hf = 0; hf < D / 64; ++hf)
+                            tma_load_4d(sRing + slot * SM::kTile + hf * SM::kHalf, map, &full[slot], hf * 64, kvh,
+                                        j * kPfKeys, b);
+                    }
+                }
+                if (*abort_flag) {   // let the copies in flight land before TMEM and smem go away
+                    mbar_wait_drain(qfull, 0, p.status);
+                    for (int i = max(0, item - kPfRing); i < item; ++i)
+                        mbar_wait_drain(&full[i % kPfRing], (i / kPfRing) & 1, p.status);
                 }
             }
-            if (*abort_flag) {   // let the copies in flight land before TMEM and smem go away
-                mbar_wait_drain(qfull, 0, p.status);
-                for (int i = max(0, item - kPfRing); i < item; ++i)
-                    mbar_wait_drain(&full[i % kPfRing], (i / kPfRing) & 1, p.status);
-            }
-        }
-        __syncwarp();
-    } else if (warp == 9) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(kPfRows, kPfKeys, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(kPfRows, D, false, true);
-            const uint32_t q_base = smem_u32(sQ);
-            const uint32_t ring_base = smem_u32(sRing);
-            auto ready = [&](int item) -> bool {
-                if (!mbar_wait(&full[item % kPfRing], (item / kPfRing) & 1, abort_flag, p.status)) return false;
-                tc_fence_after();
-                return true;
-            };
-            auto issue_qk = [&](int t, int item) {
-                const uint32_t d_tmem = tmem + t * 128;
-                const uint32_t a0 = q_base + t * SM::kTile;
-                const uint32_t b0 = ring_base + (item % kPfRing) * SM::kTile;
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint32_t o = (ks >> 2) * SM::kHalf + (ks & 3) * 32;
-                    umma_ss(d_tmem, sdesc_sw128(a0 + o, 16, 1024), sdesc_sw128(b0 + o, 16, 1024), idesc_qk, ks > 0);
-                }
-            };
-            auto issue_pv = [&](int t, int item, bool acc) {
-                const uint32_t d_tmem = tmem + 256 + t * D;
-                const uint32_t a_tmem = tmem + t * 128;
-                const uint32_t b0 = ring_base + (item % kPfRing) * SM::kTile;
-#pragma unroll
-                for (int kk = 0; kk < kPfKeys / 16; ++kk)
-                    umma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, SM::kHalf, 1024), idesc_pv,
-                            (acc || kk > 0) ? 1u : 0u);
-            };
-            bool ok = mbar_wait(qfull, 0, abort_flag, p.status) && ready(0);
-            if (ok) {
-                if (n_t0 > 0) { issue_qk(0, 0); umma_commit(&sfull[0]); }
-                if (n_t1 > 0) { issue_qk(1, 0); umma_commit(&sfull[1]); }
-                umma_commit(&empty[0]);
-            }
-            for (int j = 0; j < nmax && ok; ++j) {
-                bool v_ready = false, k_next = false;
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    const int n_t = t ? n_t1 : n_t0;
-                    if (!ok || j >= n_t) continue;
-                    if (!mbar_wait(&pfull[t], j & 1, abort_flag, p.status)) { ok = false; continue; }
+            __syncwarp();
+        } else if (warp == 9) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idesc_qk = idesc_bf16_f32(kPfRows, kPfKeys, false, false);
+                constexpr uint32_t idesc_pv = idesc_bf16_f32(kPfRows, D, false, true);
+                const uint32_t q_base = smem_u32(sQ);
+                const uint32_t ring_base = smem_u32(sRing);
+                auto ready = [&](int item) -> bool {
+                    if (!mbar_wait(&full[item % kPfRing], (item / kPfRing) & 1, abort_flag, p.status)) return false;
                     tc_fence_after();
-                    if (!v_ready) {
-                        if (!ready(2 * j + 1)) { ok = false; continue; }
-                        v_ready = true;
+                    return true;
+                };
+                auto issue_qk = [&](int t, int item) {
+                    const uint32_t d_tmem = tmem + t * 128;
+                    const uint32_t a0 = q_base + t * SM::kTile;
+                    const uint32_t b0 = ring_base + (item % kPfRing) * SM::kTile;
+    #pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t o = (ks >> 2) * SM::kHalf + (ks & 3) * 32;
+                        umma_ss(d_tmem, sdesc_sw128(a0 + o, 16, 1024), sdesc_sw128(b0 + o, 16, 1024), idesc_qk, ks > 0);
                     }
-                    issue_pv(t, 2 * j + 1, j > 0);
-                    if (j + 1 < n_t) {
-                        if (!k_next) {
-                            if (!ready(2 * j + 2)) { ok = false; continue; }
-                            k_next = true;
-                        }
-                        issue_qk(t, 2 * j + 2);
-                        umma_commit(&sfull[t]);
-                    } else {
-                        umma_commit(&odone[t]);
-                    }
+                };
+                auto issue_pv = [&](int t, int item, bool acc) {
+                    const uint32_t d_tmem = tmem + 256 + t * D;
+                    const uint32_t a_tmem = tmem + t * 128;
+                    const uint32_t b0 = ring_base + (item % kPfRing) * SM::kTile;
+    #pragma unroll
+                    for (int kk = 0; kk < kPfKeys / 16; ++kk)
+                        umma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, SM::kHalf, 1024), idesc_pv,
+                                (acc || kk > 0) ? 1u : 0u);
+                };
+                bool ok = mbar_wait(qfull, 0, abort_flag, p.status) && ready(0);
+                if (ok) {
+                    if (n_t0 > 0) { issue_qk(0, 0); umma_commit(&sfull[0]); }
+                    if (n_t1 > 0) { issue_qk(1, 0); umma_commit(&sfull[1]); }
+                    umma_commit(&empty[0]);
                 }
-                if (v_ready) umma_commit(&empty[(2 * j + 1) % kPfRing]);
-                if (k_next) umma_commit(&empty[(2 * j + 2) % kPfRing]);
+                for (int j = 0; j < nmax && ok; ++j) {
+                    bool v_ready = false, k_next = false;
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        const int n_t = t ? n_t1 : n_t0;
+                        if (!ok || j >= n_t) continue;
+                        if (!mbar_wait(&pfull[t], j & 1, abort_flag, p.status)) { ok = false; continue; }
+                        tc_fence_after();
+                        if (!v_ready) {
+                            if (!ready(2 * j + 1)) { ok = false; continue; }
+                            v_ready = true;
+                        }
+                        issue_pv(t, 2 * j + 1, j > 0);
+                        if (j + 1 < n_t) {
+                            if (!k_next) {
+                                if (!ready(2 * j + 2)) { ok = false; continue; }
+                                k_next = true;
+                            }
+                            issue_qk(t, 2 * j + 2);
+                            umma_commit(&sfull[t]);
+                        } else {
+                            umma_commit(&odone[t]);
+                        }
+                    }
+                    if (v_ready) umma_commit(&empty[(2 * j + 1) % kPfRing]);
+                    if (k_next) umma_commit(&empty[(2 * j + 2) % kPfRing]);
+                }
+                if (!ok) {   // nothing may still write TMEM when it is freed
+                    umma_commit(drain);
+                    mbar_wait_drain(drain, 0, p.status);
+                }
             }
-            if (!ok) {   // nothing may still write TMEM when it is freed
-                umma_commit(drain);
-                mbar_wait_drain(drain, 0, p.status);
-            }
+            __syncwarp();
         }
-        __syncwarp();
     } else {
+        regs_inc<kRegsSoftmax>();
         // ------------------------------------------------------------ softmax + epilogue
         const int t = warp >> 2;                    // query tile of this warpgroup
         const int quad = warp & 3;                  // TMEM lane quadrant
@@ -235,32 +245,34 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const bool landed = mbar_wait(&sfull[t], j & 1, abort_flag, p.status);
             if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }   // tcgen05.ld/st are warp-aligned
             tc_fence_after();
-            // pass 1: the row maximum (S stays in TMEM and is read again in pass
-            // 2: the 168 registers a 10-warp CTA allows cannot hold S and P)
+            // the whole S row of this thread, read once
             const int key0 = j * kPfKeys;
             const bool masked = key0 + kPfKeys - 1 > limit;
+            static_assert(kPfKeys == 128, "four 32-column TMEM loads per row");
+            uint32_t r0[32], r1[32], r2[32], r3[32];
+            tmem_ld32(tS, r0);
+            tmem_ld32(tS + 32, r1);
+            tmem_ld32(tS + 64, r2);
+            tmem_ld32(tS + 96, r3);
+            tmem_wait_ld();
+            // column c of the row (c is a compile-time constant after unrolling)
+#define GQA_S(c) ((c) < 32 ? r0[(c)] : (c) < 64 ? r1[(c) - 32] : (c) < 96 ? r2[(c) - 64] : r3[(c) - 96])
             float mx;
-            {
-                uint32_t raw[4][32];
+            if (!masked) {
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) tmem_ld32(tS + ch * 32, raw[ch]);
-                tmem_wait_ld();
-                if (!masked) {
-                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2)
-                            m4[ch] = fmax3(m4[ch], __uint_as_float(raw[ch][e]), __uint_as_float(raw[ch][e + 1]));
-                    mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-                } else {
-                    mx = -INFINITY;
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch)
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (key0 + ch * 32 + e <= limit) mx = fmaxf(mx, __uint_as_float(raw[ch][e]));
+                for (int c = 0; c < kPfKeys; c += 8) {
+                    m4[0] = fmax3(m4[0], __uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)));
+                    m4[1] = fmax3(m4[1], __uint_as_float(GQA_S(c + 2)), __uint_as_float(GQA_S(c + 3)));
+                    m4[2] = fmax3(m4[2], __uint_as_float(GQA_S(c + 4)), __uint_as_float(GQA_S(c + 5)));
+                    m4[3] = fmax3(m4[3], __uint_as_float(GQA_S(c + 6)), __uint_as_float(GQA_S(c + 7)));
                 }
+                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            } else {
+                mx = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < kPfKeys; ++c)
+                    if (key0 + c <= limit) mx = fmaxf(mx, __uint_as_float(GQA_S(c)));
             }
             const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * cl2;
             if (j == 0) {
@@ -272,49 +284,40 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     const float alpha = exp2f(m_used - m_new);
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
-                        uint32_t raw[32];
-                        tmem_ld32(tO + c * 32, raw);
+                        uint32_t ro[32];
+                        tmem_ld32(tO + c * 32, ro);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-                        tmem_st32(tO + c * 32, raw);
+                        for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
+                        tmem_st32(tO + c * 32, ro);
                     }
                     tmem_wait_st();
                     l *= alpha;
                     m_used = m_new;
                 }
             }
-            // pass 2: P = exp2(S * scale * log2(e) - m), packed bf16, written back
-            // over S; the next chunk's TMEM load is in flight while this one is
-            // computed.  The running sum adds the rounded weights.
-            float2 rs2 = make_float2(0.f, 0.f);
-            {
-                uint32_t raw[2][32];
-                tmem_ld32(tS, raw[0]);
-                tmem_wait_ld();
+            // P = exp2(S * scale * log2(e) - m) as packed bf16, written back over S;
+            // the running sum adds exactly the rounded weights P V uses
+            float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    if (ch + 1 < 4) tmem_ld32(tS + (ch + 1) * 32, raw[(ch + 1) & 1]);
-                    const uint32_t(&r)[32] = raw[ch & 1];
-                    uint32_t pk[16];
+            for (int ch = 0; ch < kPfKeys / 32; ++ch) {
+                uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float2 x = ffma2_bcast(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), cl2,
-                                                     -m_used);
-                        float a = exp2f(x.x), bb = exp2f(x.y);
-                        if (masked) {
-                            const int c = ch * 32 + 2 * e;
-                            a = (key0 + c > limit) ? 0.f : a;
-                            bb = (key0 + c + 1 > limit) ? 0.f : bb;
-                        }
-                        pk[e] = pack_bf16x2(a, bb);
-                        rs2 = fadd2(rs2, unpack_bf16x2(pk[e]));
+                for (int e = 0; e < 16; ++e) {
+                    const int c = ch * 32 + 2 * e;
+                    const float2 x = ffma2_bcast(__uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)), cl2, -m_used);
+                    uint32_t pp = pack_bf16x2(exp2f(x.x), exp2f(x.y));
+                    if (masked) {   // masked keys add nothing (also when scale == 0)
+                        if (key0 + c > limit) pp &= 0xFFFF0000u;
+                        if (key0 + c + 1 > limit) pp &= 0x0000FFFFu;
                     }
-                    tmem_st16(tS + ch * 16, pk);
-                    if (ch + 1 < 4) tmem_wait_ld();
+                    pk[e] = pp;
+                    rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(pp));
                 }
+                tmem_st16(tS + ch * 16, pk);
             }
-            const float rs = rs2.x + rs2.y;
+#undef GQA_S
+            const float rs = (rs2[0].x + rs2[1].x) + (rs2[0].y + rs2[1].y);
             l += rs;
             tmem_wait_st();
             tc_fence_before();
