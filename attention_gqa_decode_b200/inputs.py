@@ -10,6 +10,14 @@ bf16 with round-to-nearest-even.  Ragged decode lengths are integers uniform
 on a closed range, drawn by a generator seeded with the workload's seed; the
 q/k/v of each point of the ragged sweep then come from a generator seeded
 with ``seed * 1000 + n_kv``, so all points share one set of lengths.
+
+8-bit caches are made from the same bf16 draws: per KV head, a scale
+amax / 448 (the largest finite E4M3 magnitude) and codes from torch's own
+cast of value / scale to ``float8_e4m3fn`` (round to nearest even).  Paged
+caches hold the same rows as the packed ones, cut into pages of
+``page_size`` tokens whose order in memory is a seeded random permutation;
+the slots past a sequence's end, and the spare pages, are filled with NaN
+(bf16 0x7fc0, E4M3 0x7f) so that reading them would show in any result.
 """
 from __future__ import annotations
 
@@ -118,3 +126,68 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """The raw bf16 bit patterns of a CPU tensor, as a contiguous uint16 array."""
     assert t.dtype == torch.bfloat16
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+E4M3_MAX = 448.0          # largest finite magnitude of the OCP E4M3 format
+
+
+def quantize_e4m3_per_head(x: torch.Tensor):
+    """[T, n_kv, d] bf16 -> (codes uint8 [T, n_kv, d], scale float32 [n_kv]).
+
+    scale[g] = amax over head g / 448 (1 for an all-zero head); codes are
+    torch's round-to-nearest-even cast of x / scale[g] to float8_e4m3fn.
+    """
+    xf = x.to(torch.float32)
+    amax = xf.abs().amax(dim=(0, 2)) if xf.shape[0] else torch.zeros(xf.shape[1])
+    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax)).to(torch.float32)
+    codes = (xf / scale[None, :, None]).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
+    return codes.view(torch.uint8), scale
+
+
+def decode_fp8_inputs(seed: int, B: int, h: int, n_kv: int, d: int, seqlens):
+    """The draws of :func:`decode_inputs`, with both caches stored as E4M3 codes.
+
+    Returns q bf16 [B,h,d], k_codes and v_codes uint8 [sum(seqlens), n_kv, d],
+    k_scale and v_scale float32 [n_kv], seqlens int32 [B].
+    """
+    q, k, v, seqlens = decode_inputs(seed, B, h, n_kv, d, seqlens)
+    kc, ks = quantize_e4m3_per_head(k)
+    vc, vs = quantize_e4m3_per_head(v)
+    return q, kc, vc, ks, vs, seqlens
+
+
+def page_caches(seed: int, k: torch.Tensor, v: torch.Tensor, seqlens, page_size: int, spare_pages: int = 0):
+    """Cut packed caches [sum(seqlens), n_kv, d] into pages.
+
+    Returns (k_pages, v_pages [num_pages, page_size, n_kv, d], block_table
+    int32 [B, max_blocks]).  Pages are placed in a seeded random order;
+    block-table entries past a sequence's last page are -1; unused slots and
+    the ``spare_pages`` extra pages hold NaN.
+    """
+    lens = torch.as_tensor(seqlens, dtype=torch.int32).reshape(-1)
+    B = lens.numel()
+    n_blocks = [(max(int(L), 0) + page_size - 1) // page_size for L in lens.tolist()]
+    max_blocks = max(1, max(n_blocks) if n_blocks else 1)
+    num_pages = sum(n_blocks) + spare_pages
+    g = _gen(seed)
+    order = torch.randperm(max(num_pages, 1), generator=g)[:num_pages]
+    T, n_kv, d = k.shape
+    nan_code = 0x7FC0 if k.dtype == torch.bfloat16 else 0x7F
+    raw = torch.int16 if k.dtype == torch.bfloat16 else torch.uint8
+    fill = torch.tensor(nan_code, dtype=torch.int32).to(raw)
+    kp = fill.repeat(max(num_pages, 1) * page_size * n_kv * d).view(max(num_pages, 1), page_size, n_kv, d)
+    vp = kp.clone()
+    bt = torch.full((B, max_blocks), -1, dtype=torch.int32)
+    kr, vr = k.view(raw), v.view(raw)
+    row, used = 0, 0
+    for b in range(B):
+        L = max(int(lens[b]), 0)
+        for j in range(n_blocks[b]):
+            page = int(order[used])
+            used += 1
+            n = min(page_size, L - j * page_size)
+            kp[page, :n] = kr[row + j * page_size: row + j * page_size + n]
+            vp[page, :n] = vr[row + j * page_size: row + j * page_size + n]
+            bt[b, j] = page
+        row += L
+    return kp.view(k.dtype)[:num_pages], vp.view(v.dtype)[:num_pages], bt

@@ -9,7 +9,11 @@ file only compiles it with gcc, loads it with ctypes and marshals arrays.
 Every function here is pinned by ``tests/test_oracle_pins.py`` to facts the
 pages and the mathematics fix (closed forms, invariants, a brute-force
 restatement through the expand-then-reshape K/V repetition, the KV-cache
-worked number).  Parity status: pinned.
+worked number).  The 8-bit and paged decode caches (:func:`decode_general`,
+:func:`e4m3_value`) are pinned by ``tests/test_oracle_pins_cache.py``
+(torch's own E4M3 table, the brute-force restatement on torch-dequantised
+caches, the algebra of the two scales, paged == packed bit for bit).
+Parity status: pinned.
 """
 from __future__ import annotations
 
@@ -29,6 +33,7 @@ _lib = None
 _u16p = ctypes.POINTER(ctypes.c_uint16)
 _f64p = ctypes.POINTER(ctypes.c_double)
 _i32p = ctypes.POINTER(ctypes.c_int32)
+_f32p = ctypes.POINTER(ctypes.c_float)
 _int = ctypes.c_int
 
 
@@ -53,7 +58,13 @@ def _load():
             lib.oracle_decode.argtypes = [_u16p, _u16p, _u16p, _i32p, _f64p] + [_int] * 4 + [ctypes.c_double, _int]
             lib.oracle_prefill_probs.argtypes = ([_u16p, _u16p, _u16p, _f64p] + [_int] * 7 +
                                                  [ctypes.c_double, _int, _int])
-            for f in (lib.oracle_prefill, lib.oracle_prefill_rows, lib.oracle_decode, lib.oracle_prefill_probs):
+            lib.oracle_decode_general.argtypes = ([_u16p, ctypes.c_void_p, ctypes.c_void_p, _int, _f32p, _f32p,
+                                                   _i32p, _i32p, _int, _int, _int, _f64p] + [_int] * 4 +
+                                                  [ctypes.c_double, _int])
+            lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+            lib.oracle_e4m3_value.restype = ctypes.c_double
+            for f in (lib.oracle_prefill, lib.oracle_prefill_rows, lib.oracle_decode, lib.oracle_prefill_probs,
+                      lib.oracle_decode_general):
                 f.restype = _int
             _lib = lib
     return _lib
@@ -137,3 +148,72 @@ def prefill_probs(q, k, v, b: int, i: int, causal: bool = True, scale: float | N
     if rc:
         raise ValueError("oracle_prefill_probs rejected its arguments")
     return probs
+
+
+# ----------------------------------------------------------------------------
+# 8-bit (E4M3) and paged decode caches
+
+def e4m3_value(code: int) -> float:
+    """The real number an OCP E4M3 code (0..255) stands for (NaN for 0x7f / 0xff)."""
+    return float(_load().oracle_e4m3_value(int(code) & 0xFF))
+
+
+def _codes(x) -> np.ndarray:
+    """E4M3 codes as a contiguous uint8 array (from uint8 / float8_e4m3fn tensors or arrays)."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint8
+        return np.ascontiguousarray(x)
+    import torch
+    if x.dtype == torch.float8_e4m3fn:
+        x = x.view(torch.uint8)
+    assert x.dtype == torch.uint8, x.dtype
+    return np.ascontiguousarray(x.detach().cpu().contiguous().numpy())
+
+
+def _f32(x, n: int) -> np.ndarray:
+    a = np.ascontiguousarray(np.asarray(x.cpu() if hasattr(x, "cpu") else x, dtype=np.float32).reshape(n))
+    return a
+
+
+def decode_general(q, k_cache, v_cache, seqlens, *, fp8: bool = False, k_scale=None, v_scale=None,
+                   block_table=None, page_size: int = 0, scale: float | None = None,
+                   n_threads: int = 0) -> np.ndarray:
+    """One decode step over a bf16 or E4M3 cache, packed or paged; returns fp64 [B,h,d].
+
+    Packed (``block_table is None``): caches [sum(seqlens), n_kv, d] as in :func:`decode`.
+    Paged: caches [num_pages, page_size, n_kv, d]; ``block_table`` [B, max_blocks]
+    int32; token t of sequence b sits in slot t % page_size of page
+    block_table[b, t // page_size].  E4M3 caches take one fp32 scale per KV head
+    for K (``k_scale``) and one for V (``v_scale``).
+    """
+    qb = _bits(q)
+    B, h, d = qb.shape
+    if fp8:
+        kb, vb = _codes(k_cache), _codes(v_cache)
+    else:
+        kb, vb = _bits(k_cache), _bits(v_cache)
+    n_kv = kb.shape[-2]
+    lens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32).reshape(B))
+    ks = _f32(k_scale, n_kv) if fp8 else None
+    vs = _f32(v_scale, n_kv) if fp8 else None
+    if block_table is None:
+        if int(np.clip(lens, 0, None).sum()) > kb.shape[0]:
+            raise ValueError("seqlens exceed the cache rows")
+        bt, max_blocks, num_pages, page_size = None, 0, 0, 0
+    else:
+        bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32).reshape(B, -1))
+        max_blocks, num_pages = bt.shape[1], kb.shape[0]
+        if kb.shape[1] != page_size:
+            raise ValueError("paged caches must be [num_pages, page_size, n_kv, d]")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.empty((B, h, d), dtype=np.float64)
+    rc = _load().oracle_decode_general(_p(qb, _u16p), kb.ctypes.data_as(ctypes.c_void_p),
+                                       vb.ctypes.data_as(ctypes.c_void_p), int(bool(fp8)),
+                                       _p(ks, _f32p) if fp8 else None, _p(vs, _f32p) if fp8 else None,
+                                       _p(lens, _i32p), _p(bt, _i32p) if bt is not None else None,
+                                       max_blocks, page_size, num_pages, _p(out, _f64p), B, h, n_kv, d,
+                                       float(scale), n_threads)
+    if rc:
+        raise ValueError("oracle_decode_general rejected its arguments")
+    return out

@@ -20,6 +20,22 @@
  * query rows against all keys is materialised in fp64, masked, soft-maxed row
  * by row (max subtracted, as a softmax is usually evaluated), and multiplied
  * by V.  Inputs are bf16 bit patterns; each is widened exactly to fp64.
+ *
+ * Decode caches may also be stored as 8-bit floats or in pages:
+ *   "Multi-Query Attention (MQA)" (inferensys glossary), paragraph "KV cache
+ *   quantization": K and V are kept in a lower precision (FP8 among the
+ *   formats named) with scaling factors; "Multi-query attention"
+ *   (pranaymahendrakar), "Interaction with other techniques": an fp8 cache
+ *   halves the bytes per element.  Reading taken here: the OCP E4M3 format
+ *   (no infinities) with one fp32 scale per KV head for K and one for V; a
+ *   cached value is code_value * scale, widened exactly to fp64 (4 + 24
+ *   significant bits fit in 53).
+ *   Same glossary, paragraph "PagedAttention": each sequence's cache is cut
+ *   into fixed-size pages that may lie anywhere in memory.  Reading taken
+ *   here: token t of sequence b is slot t % page_size of page
+ *   block_table[b][t / page_size], a page holding [page_size, n_kv, d].
+ * Either way the cached rows are first gathered into plain fp64 K and V
+ * matrices, then the same untiled attention runs.
  */
 #include <math.h>
 #include <pthread.h>
@@ -36,23 +52,29 @@ static double bf16_value(uint16_t bits) {
 }
 
 /*
- * One attention unit.  q_rows: nr query vectors (length d, already fp64).
- * keys/vals: row j of K and V for j < nk, given as bf16 pointers with a row
- * stride in elements.  visible[r]: query row r sees keys j < visible[r].
- * out: nr x d.  probs (optional): nr x nk softmax matrix.
+ * OCP 8-bit floating point E4M3 (the variant without infinities): sign bit,
+ * 4 exponent bits with bias 7, 3 mantissa bits.  Exponent field 0 encodes the
+ * subnormals (m / 8) * 2^-6; exponent 15 with mantissa 7 is NaN; every other
+ * code is (1 + m / 8) * 2^(e - 7), so the largest finite magnitude is 448.
  */
-static int attend(const double *q_rows, int nr, const uint16_t *k0, const uint16_t *v0,
-                  long kv_row_stride, int nk, int d, const int *visible, double scale,
-                  double *out, double *probs) {
+double oracle_e4m3_value(uint8_t code) {
+    int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m / 8.0, -6);
+    else mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+/*
+ * One attention unit on fp64 operands.  q_rows: nr query vectors of length d.
+ * kd/vd: nk x d keys and values.  visible[r]: query row r sees keys
+ * j < visible[r].  out: nr x d.  probs (optional): nr x nk softmax matrix.
+ */
+static int attend_f64(const double *q_rows, int nr, const double *kd, const double *vd, int nk, int d,
+                      const int *visible, double scale, double *out, double *probs) {
     double *S = (double *)malloc(sizeof(double) * (size_t)(nr > 0 ? nr : 1) * (size_t)(nk > 0 ? nk : 1));
-    double *kd = (double *)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1) * (size_t)d);
-    double *vd = (double *)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1) * (size_t)d);
-    if (!S || !kd || !vd) { free(S); free(kd); free(vd); return -1; }
-    for (int j = 0; j < nk; ++j)
-        for (int c = 0; c < d; ++c) {
-            kd[(size_t)j * d + c] = bf16_value(k0[(size_t)j * kv_row_stride + c]);
-            vd[(size_t)j * d + c] = bf16_value(v0[(size_t)j * kv_row_stride + c]);
-        }
+    if (!S) return -1;
     /* scores, with the mask */
     for (int r = 0; r < nr; ++r)
         for (int j = 0; j < nk; ++j) {
@@ -86,8 +108,25 @@ static int attend(const double *q_rows, int nr, const uint16_t *k0, const uint16
             for (int c = 0; c < d; ++c) orow[c] += p * vd[(size_t)j * d + c];
         }
     }
-    free(S); free(kd); free(vd);
+    free(S);
     return 0;
+}
+
+/* The same unit with bf16 K/V rows read through a row stride (in elements). */
+static int attend(const double *q_rows, int nr, const uint16_t *k0, const uint16_t *v0,
+                  long kv_row_stride, int nk, int d, const int *visible, double scale,
+                  double *out, double *probs) {
+    double *kd = (double *)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1) * (size_t)d);
+    double *vd = (double *)malloc(sizeof(double) * (size_t)(nk > 0 ? nk : 1) * (size_t)d);
+    if (!kd || !vd) { free(kd); free(vd); return -1; }
+    for (int j = 0; j < nk; ++j)
+        for (int c = 0; c < d; ++c) {
+            kd[(size_t)j * d + c] = bf16_value(k0[(size_t)j * kv_row_stride + c]);
+            vd[(size_t)j * d + c] = bf16_value(v0[(size_t)j * kv_row_stride + c]);
+        }
+    int rc = attend_f64(q_rows, nr, kd, vd, nk, d, visible, scale, out, probs);
+    free(kd); free(vd);
+    return rc;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -98,6 +137,12 @@ typedef struct {
     const uint16_t *q, *k, *v;
     const int32_t *seqlens;
     const long *offsets;      /* decode: first cache row of each sequence */
+    /* general decode (kind 2): cache element format and page table */
+    const void *kc, *vc;      /* caches: bf16 bits (fmt 0) or E4M3 codes (fmt 1) */
+    int fmt;
+    const float *k_scale, *v_scale;   /* fmt 1: one scale per KV head */
+    const int32_t *block_table;       /* NULL: packed layout */
+    int max_blocks, page_size;
     double *out;
     int B, S_q, S_kv, h, n_kv, d, causal;
     double scale;
@@ -155,12 +200,51 @@ static void run_decode_unit(job_t *J, int b, int i) {
     free(qd);
 }
 
+/* Cache row of token t of sequence b (in units of n_kv * d elements). */
+static long cache_row(const job_t *J, int b, int t) {
+    if (!J->block_table) return J->offsets[b] + t;
+    int page = J->block_table[(size_t)b * J->max_blocks + t / J->page_size];
+    return (long)page * J->page_size + t % J->page_size;
+}
+
+static double cache_value(const job_t *J, const void *cache, const float *sc, long idx, int g) {
+    if (J->fmt == 0) return bf16_value(((const uint16_t *)cache)[idx]);
+    return oracle_e4m3_value(((const uint8_t *)cache)[idx]) * (double)sc[g];
+}
+
+static void run_decode_general_unit(job_t *J, int b, int i) {
+    int G = J->h / J->n_kv;
+    int g = i / G;
+    int d = J->d;
+    int L = J->seqlens[b];
+    double *orow = J->out + ((size_t)b * J->h + i) * d;
+    if (L <= 0) { for (int c = 0; c < d; ++c) orow[c] = 0.0; return; }
+    double *qd = (double *)malloc(sizeof(double) * (size_t)d);
+    double *kd = (double *)malloc(sizeof(double) * (size_t)L * d);
+    double *vd = (double *)malloc(sizeof(double) * (size_t)L * d);
+    if (!qd || !kd || !vd) { free(qd); free(kd); free(vd); J->failed = 1; return; }
+    const uint16_t *qrow = J->q + ((size_t)b * J->h + i) * d;
+    for (int c = 0; c < d; ++c) qd[c] = bf16_value(qrow[c]);
+    /* gather the cached rows of KV head g */
+    for (int t = 0; t < L; ++t) {
+        long base = (cache_row(J, b, t) * J->n_kv + g) * (long)d;
+        for (int c = 0; c < d; ++c) {
+            kd[(size_t)t * d + c] = cache_value(J, J->kc, J->k_scale, base + c, g);
+            vd[(size_t)t * d + c] = cache_value(J, J->vc, J->v_scale, base + c, g);
+        }
+    }
+    if (attend_f64(qd, 1, kd, vd, L, d, &L, J->scale, orow, NULL)) J->failed = 1;
+    free(qd); free(kd); free(vd);
+}
+
 static void *worker(void *p) {
     worker_arg_t *a = (worker_arg_t *)p;
     job_t *J = a->job;
     for (int u = a->tid; u < J->n_units; u += J->n_threads) {
         if (J->kind == 1) {
             run_decode_unit(J, u / J->h, u % J->h);
+        } else if (J->kind == 2) {
+            run_decode_general_unit(J, u / J->h, u % J->h);
         } else if (J->sample) {
             const int32_t *s = J->sample + 3 * (size_t)u;
             int r = s[2];
@@ -281,5 +365,47 @@ int oracle_prefill_probs(const uint16_t *q, const uint16_t *k, const uint16_t *v
     int rc = attend(qd, S_q, k + ((size_t)b * S_kv * n_kv + g) * d, v + ((size_t)b * S_kv * n_kv + g) * d,
                     (long)n_kv * d, S_kv, d, vis, scale, o, probs);
     free(qd); free(o); free(vis);
+    return rc;
+}
+
+/* One decode step over a cache in either element format and either layout.
+ *   fmt 0: k_cache/v_cache hold bf16 bits; fmt 1: E4M3 codes, the value of
+ *          a code of KV head g being oracle_e4m3_value(code) * k_scale[g]
+ *          (resp. v_scale[g]).
+ *   block_table == NULL: packed caches [sum(max(seqlens,0)), n_kv, d], as in
+ *          oracle_decode.  Otherwise paged caches [num_pages, page_size, n_kv, d]
+ *          and block_table [B, max_blocks]: token t of sequence b is slot
+ *          t % page_size of page block_table[b * max_blocks + t / page_size].
+ * Returns -1 for bad shapes, a page index outside [0, num_pages) or a length
+ * beyond max_blocks * page_size. */
+int oracle_decode_general(const uint16_t *q, const void *k_cache, const void *v_cache, int fmt,
+                          const float *k_scale, const float *v_scale, const int32_t *seqlens,
+                          const int32_t *block_table, int max_blocks, int page_size, int num_pages,
+                          double *out, int B, int h, int n_kv, int d, double scale, int n_threads) {
+    if (!check_shape(B, h, n_kv, d) || (fmt != 0 && fmt != 1)) return -1;
+    if (fmt == 1 && (!k_scale || !v_scale)) return -1;
+    long *off = (long *)malloc(sizeof(long) * (size_t)B);
+    if (!off) return -1;
+    long acc = 0;
+    for (int b = 0; b < B; ++b) { off[b] = acc; if (seqlens[b] > 0) acc += seqlens[b]; }
+    if (block_table) {
+        if (max_blocks <= 0 || page_size <= 0 || num_pages <= 0) { free(off); return -1; }
+        for (int b = 0; b < B; ++b) {
+            int L = seqlens[b];
+            if (L > (long)max_blocks * page_size) { free(off); return -1; }
+            for (int t = 0; t < L; t += page_size) {
+                int page = block_table[(size_t)b * max_blocks + t / page_size];
+                if (page < 0 || page >= num_pages) { free(off); return -1; }
+            }
+        }
+    }
+    job_t J = {0};
+    J.kind = 2; J.q = q; J.kc = k_cache; J.vc = v_cache; J.fmt = fmt;
+    J.k_scale = k_scale; J.v_scale = v_scale; J.seqlens = seqlens; J.offsets = off;
+    J.block_table = block_table; J.max_blocks = max_blocks; J.page_size = page_size;
+    J.out = out; J.B = B; J.h = h; J.n_kv = n_kv; J.d = d; J.scale = scale;
+    J.n_units = B * h;
+    int rc = run_job(&J, n_threads);
+    free(off);
     return rc;
 }
