@@ -7,8 +7,10 @@ current CUDA stream, and raises on any non-zero status.  PyTorch is used only
 for device memory and streams.  There is no CPU fallback: if the library is
 missing, importing the binding's entry points fails loudly.
 """
-from ._lib import (GQAError, decode, gqa_decode, gqa_get_device_status, gqa_prefill,  # noqa: F401
-                   gqa_status_string, lib, library_path, prefill)
+from ._lib import (GQAError, decode, decode_fp8, decode_paged, gqa_decode, gqa_decode_fp8,  # noqa: F401
+                   gqa_decode_paged, gqa_decode_paged_fp8, gqa_get_device_status, gqa_prefill, gqa_status_string,
+                   lib, library_path, prefill)
 
-__all__ = ["prefill", "decode", "gqa_prefill", "gqa_decode", "gqa_status_string", "gqa_get_device_status",
+__all__ = ["prefill", "decode", "decode_fp8", "decode_paged", "gqa_prefill", "gqa_decode", "gqa_decode_fp8",
+           "gqa_decode_paged", "gqa_decode_paged_fp8", "gqa_status_string", "gqa_get_device_status",
            "GQAError", "lib", "library_path"]

@@ -18,6 +18,9 @@ _vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "gqa_prefill": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
+    "gqa_decode_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
+    "gqa_decode_paged": ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
+    "gqa_decode_paged_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_status_string": ([_i], ctypes.c_char_p),
     "gqa_get_device_status": ([_vp], _i),
 }
@@ -68,6 +71,23 @@ def gqa_prefill(q, k, v, out, B, S_q, S_kv, h, n_kv, d_h, causal, scale, stream)
 
 def gqa_decode(q, k_cache, v_cache, seqlens, out, B, h, n_kv, d_h, scale, stream) -> int:
     return lib().gqa_decode(q, k_cache, v_cache, seqlens, out, B, h, n_kv, d_h, float(scale), stream)
+
+
+def gqa_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, B, h, n_kv, d_h, scale, stream) -> int:
+    return lib().gqa_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, B, h, n_kv, d_h,
+                                float(scale), stream)
+
+
+def gqa_decode_paged(q, k_pages, v_pages, block_table, max_blocks, page_size, num_pages, seqlens, out,
+                     B, h, n_kv, d_h, scale, stream) -> int:
+    return lib().gqa_decode_paged(q, k_pages, v_pages, block_table, max_blocks, page_size, num_pages, seqlens,
+                                  out, B, h, n_kv, d_h, float(scale), stream)
+
+
+def gqa_decode_paged_fp8(q, k_pages, v_pages, k_scale, v_scale, block_table, max_blocks, page_size, num_pages,
+                         seqlens, out, B, h, n_kv, d_h, scale, stream) -> int:
+    return lib().gqa_decode_paged_fp8(q, k_pages, v_pages, k_scale, v_scale, block_table, max_blocks, page_size,
+                                      num_pages, seqlens, out, B, h, n_kv, d_h, float(scale), stream)
 
 
 def gqa_get_device_status(stream=None) -> int:
@@ -145,4 +165,116 @@ def decode(q, k_cache, v_cache, seqlens, scale: float | None = None, out=None, s
                         B, h, n_kv, d, scale, _stream_ptr(stream))
     if st != GQA_OK:
         raise GQAError(st, "gqa_decode")
+    return out
+
+
+def _check_cache(t, name, ndim, fp8):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    want = (torch.uint8, torch.float8_e4m3fn) if fp8 else (torch.bfloat16,)
+    if t.dtype not in want:
+        raise TypeError(f"{name} must be {' or '.join(map(str, want))}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check_scales(k_scale, v_scale, n_kv):
+    import torch
+    for name, t in (("k_scale", k_scale), ("v_scale", v_scale)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or not t.is_cuda \
+                or t.numel() != n_kv or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous float32 CUDA tensor with n_kv = {n_kv} entries")
+
+
+def _check_seqlens(seqlens, B):
+    import torch
+    if not isinstance(seqlens, torch.Tensor) or seqlens.dtype != torch.int32 or not seqlens.is_cuda \
+            or seqlens.numel() != B or not seqlens.is_contiguous():
+        raise ValueError("seqlens must be a contiguous int32 CUDA tensor with B entries")
+
+
+def decode_fp8(q, k_cache, v_cache, k_scale, v_scale, seqlens, scale: float | None = None, out=None,
+               stream=None):
+    """One decode step over packed E4M3 caches [sum(seqlens), n_kv, d] (uint8 codes or float8_e4m3fn).
+
+    The value of a cached code of KV head g is code * k_scale[g] (K) or
+    code * v_scale[g] (V); the scales are float32 [n_kv] CUDA tensors.  q is
+    bf16 [B, h, d]; returns bf16 [B, h, d].
+    """
+    import torch
+    _check_cache(k_cache, "k_cache", 3, True), _check_cache(v_cache, "v_cache", 3, True)
+    _check(q, "q", 3)
+    B, h, d = q.shape
+    T, n_kv, dk = k_cache.shape
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or dk != d:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k_cache.shape)} v{tuple(v_cache.shape)}")
+    _check_scales(k_scale, v_scale, n_kv)
+    _check_seqlens(seqlens, B)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check(out, "out", 3)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    with torch.cuda.device(q.device):
+        st = gqa_decode_fp8(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), k_scale.data_ptr(),
+                            v_scale.data_ptr(), seqlens.data_ptr(), out.data_ptr(), B, h, n_kv, d, scale,
+                            _stream_ptr(stream))
+    if st != GQA_OK:
+        raise GQAError(st, "gqa_decode_fp8")
+    return out
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale: float | None = None, k_scale=None,
+                 v_scale=None, out=None, stream=None):
+    """One decode step over paged caches [num_pages, page_size, n_kv, d].
+
+    Token t of sequence b is slot t % page_size of page block_table[b, t // page_size]
+    (block_table: int32 [B, max_blocks] CUDA tensor).  bf16 pages, or E4M3
+    pages (uint8 / float8_e4m3fn) with ``k_scale`` and ``v_scale`` float32 [n_kv].
+    page_size must be a power of two in [16, 65536].  Returns bf16 [B, h, d].
+    """
+    import torch
+    fp8 = k_pages.dtype in (torch.uint8, torch.float8_e4m3fn)
+    _check(q, "q", 3)
+    _check_cache(k_pages, "k_pages", 4, fp8), _check_cache(v_pages, "v_pages", 4, fp8)
+    B, h, d = q.shape
+    num_pages, page_size, n_kv, dk = k_pages.shape
+    if tuple(v_pages.shape) != tuple(k_pages.shape) or dk != d:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k_pages.shape)} v{tuple(v_pages.shape)}")
+    if not isinstance(block_table, torch.Tensor) or block_table.dtype != torch.int32 or not block_table.is_cuda \
+            or block_table.dim() != 2 or block_table.shape[0] != B or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous int32 CUDA tensor [B, max_blocks]")
+    _check_seqlens(seqlens, B)
+    if fp8:
+        _check_scales(k_scale, v_scale, n_kv)
+    elif k_scale is not None or v_scale is not None:
+        raise ValueError("scales apply to E4M3 pages only")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check(out, "out", 3)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    mb = block_table.shape[1]
+    with torch.cuda.device(q.device):
+        if fp8:
+            st = gqa_decode_paged_fp8(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), k_scale.data_ptr(),
+                                      v_scale.data_ptr(), block_table.data_ptr(), mb, page_size, num_pages,
+                                      seqlens.data_ptr(), out.data_ptr(), B, h, n_kv, d, scale, _stream_ptr(stream))
+        else:
+            st = gqa_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(), mb,
+                                  page_size, num_pages, seqlens.data_ptr(), out.data_ptr(), B, h, n_kv, d, scale,
+                                  _stream_ptr(stream))
+    if st != GQA_OK:
+        raise GQAError(st, "gqa_decode_paged_fp8" if fp8 else "gqa_decode_paged")
     return out

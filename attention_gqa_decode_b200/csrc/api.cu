@@ -14,6 +14,9 @@ int launch_prefill(const void *q, const void *k, const void *v, void *out, int B
                    int d, int causal, float scale, cudaStream_t stream);
 int launch_decode(const void *q, const void *k, const void *v, const int32_t *seqlens, void *out, int B, int h,
                   int n_kv, int d, float scale, cudaStream_t stream);
+int launch_decode_ex(const void *q, const void *k, const void *v, const float *k_scale, const float *v_scale,
+                     const int32_t *seqlens, const int32_t *block_table, int max_blocks, int page_size,
+                     int num_pages, void *out, int B, int h, int n_kv, int d, float scale, cudaStream_t stream);
 }  // namespace gqa
 
 namespace gqa_host {
@@ -33,6 +36,13 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool encode_tensor_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
                        const uint64_t *strides_bytes, const uint32_t *box) {
+    return encode_tensor_map_ex(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_128B, base, rank, dims,
+                                strides_bytes, box);
+}
+
+bool encode_tensor_map_ex(CUtensorMap *map, CUtensorMapDataType dtype, CUtensorMapSwizzle swizzle,
+                          const void *base, int rank, const uint64_t *dims, const uint64_t *strides_bytes,
+                          const uint32_t *box) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t gdim[5];
@@ -44,8 +54,8 @@ bool encode_tensor_map(CUtensorMap *map, const void *base, int rank, const uint6
         estride[i] = 1;
         if (i + 1 < rank) gstride[i] = strides_bytes[i];
     }
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void *>(base),
-                    gdim, gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    CUresult r = fn(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void *>(base),
+                    gdim, gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -102,6 +112,72 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
     if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
     if (static_cast<long>(n_kv) * ((h / n_kv + 63) / 64) > 65535) return GQA_ERR_UNSUPPORTED;
     return gqa::launch_decode(q, k_cache, v_cache, seqlens, out, B, h, n_kv, d_h, scale, stream);
+}
+
+// Checks shared by every decode entry point (cache pointers are checked by the caller).
+static int decode_args_ok(const void *q, const int32_t *seqlens, const void *out, int B, int h, int n_kv, int d_h,
+                          float scale) {
+    if (!q || !seqlens || !out) return GQA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return GQA_ERR_INVALID_ARG;
+    if (B <= 0 || B > 65535 || h <= 0 || n_kv <= 0 || h % n_kv != 0) return GQA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return GQA_ERR_INVALID_ARG;
+    if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
+    if (static_cast<long>(n_kv) * ((h / n_kv + 63) / 64) > 65535) return GQA_ERR_UNSUPPORTED;
+    return GQA_OK;
+}
+
+static int caches_ok(const void *k, const void *v) {
+    return (k && v && aligned16(k) && aligned16(v)) ? GQA_OK : GQA_ERR_INVALID_ARG;
+}
+
+static int scales_ok(const float *k_scale, const float *v_scale) {
+    if (!k_scale || !v_scale) return GQA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+        return GQA_ERR_INVALID_ARG;
+    return GQA_OK;
+}
+
+static int pages_ok(const int32_t *block_table, int max_blocks, int page_size, int num_pages) {
+    if (!block_table || (reinterpret_cast<uintptr_t>(block_table) & 3u)) return GQA_ERR_INVALID_ARG;
+    if (max_blocks <= 0 || num_pages <= 0) return GQA_ERR_INVALID_ARG;
+    if (page_size < 16 || page_size > 65536 || (page_size & (page_size - 1))) return GQA_ERR_INVALID_ARG;
+    if (static_cast<long long>(max_blocks) * page_size > 0x7FFFFFFFLL) return GQA_ERR_INVALID_ARG;
+    return GQA_OK;
+}
+
+int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, const float *k_scale,
+                   const float *v_scale, const int32_t *seqlens, void *out, int B, int h, int n_kv, int d_h,
+                   float scale, cudaStream_t stream) {
+    int st = caches_ok(k_cache, v_cache);
+    if (st == GQA_OK) st = scales_ok(k_scale, v_scale);
+    if (st == GQA_OK) st = decode_args_ok(q, seqlens, out, B, h, n_kv, d_h, scale);
+    if (st != GQA_OK) return st;
+    return gqa::launch_decode_ex(q, k_cache, v_cache, k_scale, v_scale, seqlens, nullptr, 0, 0, 0, out, B, h, n_kv,
+                                 d_h, scale, stream);
+}
+
+int gqa_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int32_t *block_table,
+                     int max_blocks, int page_size, int num_pages, const int32_t *seqlens, void *out, int B, int h,
+                     int n_kv, int d_h, float scale, cudaStream_t stream) {
+    int st = caches_ok(k_pages, v_pages);
+    if (st == GQA_OK) st = pages_ok(block_table, max_blocks, page_size, num_pages);
+    if (st == GQA_OK) st = decode_args_ok(q, seqlens, out, B, h, n_kv, d_h, scale);
+    if (st != GQA_OK) return st;
+    return gqa::launch_decode_ex(q, k_pages, v_pages, nullptr, nullptr, seqlens, block_table, max_blocks, page_size,
+                                 num_pages, out, B, h, n_kv, d_h, scale, stream);
+}
+
+int gqa_decode_paged_fp8(const void *q, const void *k_pages, const void *v_pages, const float *k_scale,
+                         const float *v_scale, const int32_t *block_table, int max_blocks, int page_size,
+                         int num_pages, const int32_t *seqlens, void *out, int B, int h, int n_kv, int d_h,
+                         float scale, cudaStream_t stream) {
+    int st = caches_ok(k_pages, v_pages);
+    if (st == GQA_OK) st = scales_ok(k_scale, v_scale);
+    if (st == GQA_OK) st = pages_ok(block_table, max_blocks, page_size, num_pages);
+    if (st == GQA_OK) st = decode_args_ok(q, seqlens, out, B, h, n_kv, d_h, scale);
+    if (st != GQA_OK) return st;
+    return gqa::launch_decode_ex(q, k_pages, v_pages, k_scale, v_scale, seqlens, block_table, max_blocks, page_size,
+                                 num_pages, out, B, h, n_kv, d_h, scale, stream);
 }
 
 const char *gqa_status_string(int status) {

@@ -7,6 +7,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -16,6 +18,7 @@ namespace gqa {
 // The device status word (one int per device, owned by the library) is passed
 // to every kernel; the first error a kernel records wins, and the host reads
 // and clears it through gqa_get_device_status().
+constexpr int kStatusInvalid = 1;   // == GQA_ERR_INVALID_ARG (a bad value found on the device)
 constexpr int kStatusTimeout = 4;   // == GQA_ERR_TIMEOUT
 
 // A wait gives up after this many nanoseconds of global time (about a second).
@@ -31,9 +34,9 @@ __device__ __forceinline__ unsigned long long global_ns() {
     return t;
 }
 
-__device__ __forceinline__ void record_timeout(int *status) {
-    atomicCAS(status, 0, kStatusTimeout);
-}
+__device__ __forceinline__ void record_status(int *status, int code) { atomicCAS(status, 0, code); }
+
+__device__ __forceinline__ void record_timeout(int *status) { record_status(status, kStatusTimeout); }
 
 // ---------------------------------------------------------------------------
 // mbarrier
@@ -154,6 +157,45 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
         "{%0, %1, %2, %3};"
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The same with f16 operands (fp32 accumulate).
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Transpose of an 8x8 matrix of 16-bit elements held one row pair per lane
+// (lane l: row l / 4, columns 2 (l % 4) and 2 (l % 4) + 1) into the same layout.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);   // .x (low half) = lo
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
+    return __half22float2(*reinterpret_cast<const __half2 *>(&v));
+}
+
+// Two E4M3 codes (low byte -> low half) widened to an f16 pair.  Exact: every
+// finite E4M3 value, subnormals included, is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xFFFFu), __NV_E4M3);
+    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+// A bf16 pair re-encoded as an f16 pair (round to nearest even; exact for
+// magnitudes in [2^-14, 65504]).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+    return pack_f16x2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -343,6 +385,11 @@ namespace gqa_host {
 // driver entry point is missing or the encoding is rejected.
 bool encode_tensor_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
                        const uint64_t *strides_bytes, const uint32_t *box);
+
+// The same for another element type and swizzle mode.
+bool encode_tensor_map_ex(CUtensorMap *map, CUtensorMapDataType dtype, CUtensorMapSwizzle swizzle,
+                          const void *base, int rank, const uint64_t *dims, const uint64_t *strides_bytes,
+                          const uint32_t *box);
 
 int sm_count();
 

@@ -16,8 +16,10 @@
  *     to device memory (online softmax with a running max and running sum).
  *
  * Conventions shared by every entry point
- *   - All tensor pointers are DEVICE pointers to bf16 (IEEE bfloat16) data,
- *     row-major, 16-byte aligned, owned by the caller.  The library keeps no
+ *   - All tensor pointers are DEVICE pointers, row-major, 16-byte aligned,
+ *     owned by the caller; q/k/v/out are bf16 (IEEE bfloat16) unless an entry
+ *     point says otherwise (8-bit caches, int32 lengths and page tables,
+ *     float32 scales).  The library keeps no
  *     pointer after the call returns, allocates no device memory and creates
  *     no stream.
  *   - Work is enqueued asynchronously on `stream` (0 = legacy default stream).
@@ -99,13 +101,75 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
                const int32_t *seqlens, void *out,
                int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
 
+/*
+ * Decode over an 8-bit cache ("Multi-Query Attention (MQA)" (inferensys
+ * glossary), "KV cache quantization": the cache is kept in FP8 with scaling
+ * factors; "Multi-query attention" (pranaymahendrakar), "Interaction with
+ * other techniques": fp8 halves the bytes per cached element).
+ *   k_cache, v_cache  [sum_b seqlens[b], n_kv, d_h]  uint8   OCP E4M3 codes
+ *                     (the variant without infinities; 0x7f / 0xff are NaN),
+ *                     packed exactly as in gqa_decode
+ *   k_scale, v_scale  [n_kv]  float32  DEVICE arrays: the cached value of a
+ *                     code of KV head g is code * k_scale[g] (keys) or
+ *                     code * v_scale[g] (values)
+ *   q, seqlens, out   as in gqa_decode (bf16 q and out)
+ * The products run with f16 operands: Q is rounded to f16 (exact for
+ * magnitudes in [2^-14, 65504]; larger ones overflow) and the softmax weights
+ * are rounded to f16; the codes are exact in f16.  Accumulation is fp32.
+ * Scales must be finite and >= 0; any other value is recorded as
+ * GQA_ERR_INVALID_ARG in the device status word (gqa_get_device_status) and
+ * the affected rows are unspecified.
+ * Errors: as gqa_decode, plus GQA_ERR_INVALID_ARG for a null or
+ * non-4-byte-aligned scale pointer.
+ */
+int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache,
+                   const float *k_scale, const float *v_scale,
+                   const int32_t *seqlens, void *out,
+                   int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
+
+/*
+ * Decode over a paged bf16 cache ("Multi-Query Attention (MQA)" (inferensys
+ * glossary), "PagedAttention": each sequence's cache is cut into fixed-size
+ * pages that may lie anywhere in device memory).
+ *   k_pages, v_pages  [num_pages, page_size, n_kv, d_h]  bf16
+ *   block_table       [B, max_blocks]  int32  DEVICE array: token t of
+ *                     sequence b is slot t % page_size of page
+ *                     block_table[b * max_blocks + t / page_size]; entries
+ *                     past a sequence's last page are never read
+ *   seqlens           [B]  int32  DEVICE array, tokens per sequence (<= 0:
+ *                     zero row)
+ *   q, out            [B, h, d_h]  bf16
+ * page_size is a power of two in [16, 65536].  Slots of a page past the
+ * sequence's end may hold anything (NaN included): they are never used.
+ * A page id outside [0, num_pages), or a length above max_blocks * page_size,
+ * is recorded as GQA_ERR_INVALID_ARG in the device status word; such pages
+ * read as zeros and such lengths are cut to max_blocks * page_size.
+ * Errors: as gqa_decode, plus GQA_ERR_INVALID_ARG for a null or misaligned
+ * block_table, max_blocks or num_pages <= 0, a page_size that is not a power
+ * of two in [16, 65536], or max_blocks * page_size above INT32_MAX.
+ */
+int gqa_decode_paged(const void *q, const void *k_pages, const void *v_pages,
+                     const int32_t *block_table, int max_blocks, int page_size, int num_pages,
+                     const int32_t *seqlens, void *out,
+                     int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
+
+/* Paged E4M3 pages [num_pages, page_size, n_kv, d_h] (uint8 codes) with the
+ * per-KV-head scales of gqa_decode_fp8; everything else as gqa_decode_paged. */
+int gqa_decode_paged_fp8(const void *q, const void *k_pages, const void *v_pages,
+                         const float *k_scale, const float *v_scale,
+                         const int32_t *block_table, int max_blocks, int page_size, int num_pages,
+                         const int32_t *seqlens, void *out,
+                         int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
+
 /* A static, human-readable name for a gqa_status_t value. */
 const char *gqa_status_string(int status);
 
 /*
  * Synchronises `stream`, then returns and clears the library's device status
- * word for the current device: GQA_OK, or GQA_ERR_TIMEOUT if a kernel gave up
- * on an internal wait since the last call.  Returns GQA_ERR_CUDA if the
+ * word for the current device: GQA_OK, GQA_ERR_TIMEOUT if a kernel gave up
+ * on an internal wait since the last call, or GQA_ERR_INVALID_ARG if a kernel
+ * met a bad value that lives on the device (a page id, a length beyond the
+ * block table, a negative or non-finite cache scale).  The first error wins.  Returns GQA_ERR_CUDA if the
  * synchronisation itself fails.
  */
 int gqa_get_device_status(cudaStream_t stream);

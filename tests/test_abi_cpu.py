@@ -87,3 +87,47 @@ def test_binding_rejects_cpu_tensors():
         gqa.prefill(q, q[:, :, :1].contiguous(), q[:, :, :1].contiguous())
     with pytest.raises(TypeError):
         gqa.prefill(q.float(), q, q)
+
+
+@pytest.mark.parametrize("args,expect", [
+    # q, k, v, k_scale, v_scale, seqlens, out, B, h, n_kv, d, scale
+    ((A, A, A, A, A, A, A, 2, 4, 2, 128, 0.1), None),
+    ((A, A, A, 0, A, A, A, 2, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),      # null k_scale
+    ((A, A, A, A, A + 2, A, A, 2, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),  # misaligned v_scale
+    ((A, BAD, A, A, A, A, A, 2, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, A, A, A, 2, 4, 3, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, A, A, A, 2, 4, 2, 128, -1.0), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, A, A, A, 2, 4, 2, 96, 0.1), _lib.GQA_ERR_UNSUPPORTED),
+])
+def test_decode_fp8_rejects(L, args, expect):
+    if expect is None:
+        return   # a valid call would launch; covered by the GPU tests
+    assert gqa.gqa_decode_fp8(*args, None) == expect
+
+
+@pytest.mark.parametrize("table,mb,ps,npg,expect", [
+    (0, 4, 64, 10, _lib.GQA_ERR_INVALID_ARG),          # null block table
+    (A + 2, 4, 64, 10, _lib.GQA_ERR_INVALID_ARG),      # misaligned block table
+    (A, 0, 64, 10, _lib.GQA_ERR_INVALID_ARG),          # max_blocks = 0
+    (A, 4, 64, 0, _lib.GQA_ERR_INVALID_ARG),           # no pages
+    (A, 4, 48, 10, _lib.GQA_ERR_INVALID_ARG),          # not a power of two
+    (A, 4, 8, 10, _lib.GQA_ERR_INVALID_ARG),           # below 16
+    (A, 4, 131072, 10, _lib.GQA_ERR_INVALID_ARG),      # above 65536
+    (A, 1 << 20, 65536, 10, _lib.GQA_ERR_INVALID_ARG),  # max_blocks * page_size overflows int32
+])
+def test_decode_paged_rejects(L, table, mb, ps, npg, expect):
+    assert gqa.gqa_decode_paged(A, A, A, table, mb, ps, npg, A, A, 2, 4, 2, 128, 0.1, None) == expect
+    assert gqa.gqa_decode_paged_fp8(A, A, A, A, A, table, mb, ps, npg, A, A, 2, 4, 2, 128, 0.1, None) == expect
+
+
+def test_decode_paged_fp8_needs_scales(L):
+    assert gqa.gqa_decode_paged_fp8(A, A, A, 0, A, A, 4, 64, 10, A, A, 2, 4, 2, 128, 0.1, None) == \
+        _lib.GQA_ERR_INVALID_ARG
+
+
+def test_binding_rejects_bad_cache_dtypes():
+    import torch
+    q = torch.zeros(2, 4, 64, dtype=torch.bfloat16)
+    k = torch.zeros(8, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):       # bf16 codes for an 8-bit cache
+        gqa.decode_fp8(q, k, k, None, None, None)
