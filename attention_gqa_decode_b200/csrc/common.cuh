@@ -8,7 +8,6 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -185,11 +184,19 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t v) {
     return __half22float2(*reinterpret_cast<const __half2 *>(&v));
 }
 
-// Two E4M3 codes (low byte -> low half) widened to an f16 pair.  Exact: every
-// finite E4M3 value, subnormals included, is an f16 value.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xFFFFu), __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// Two E4M3 codes widened to an f16 pair (the lower-addressed code to the low
+// half): the low two bytes of `codes` (..._lo) or the high two (..._hi).
+// Exact: every finite E4M3 value, subnormals included, is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_lo(uint32_t codes) {
+    uint32_t d;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\t}" : "=r"(d) : "r"(codes));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_hi(uint32_t codes) {
+    uint32_t d;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, h;\n\t}" : "=r"(d) : "r"(codes));
+    return d;
 }
 
 // A bf16 pair re-encoded as an f16 pair (round to nearest even; exact for

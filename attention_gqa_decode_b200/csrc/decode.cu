@@ -57,12 +57,10 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 
-#ifndef GQA_DECODE_CTAS_PER_SM
-#define GQA_DECODE_CTAS_PER_SM 2   // resident CTAs per SM (shared memory allows two)
-#endif
 #ifndef GQA_DECODE_MAX_SPLIT
 #define GQA_DECODE_MAX_SPLIT 8     // splits per (sequence, KV head) = thread-block cluster size
 #endif
@@ -83,7 +81,7 @@ enum class KvFmt { kBf16, kE4m3 };
 template <int D, KvFmt F>
 struct DecGeom {
     static constexpr bool kFp8 = (F == KvFmt::kE4m3);
-    static constexpr int kTok = kFp8 ? 128 : 64;         // tokens per pipeline stage
+    static constexpr int kTok = kFp8 ? 128 : 64;         // tokens per pipeline stage (16 KB of K at d = 128)
     static constexpr int kRowBytes = kFp8 ? D : 128;     // one token's bytes in a panel
     static constexpr int kPanels = kFp8 ? 1 : D / 64;
     static constexpr int kBoxInner = kFp8 ? D : 64;      // TMA box, innermost extent in elements
@@ -109,7 +107,7 @@ struct DecodeParams {
     int *status;                      // the library's device status word
 };
 
-template <int D, KvFmt F, int STAGES>
+template <int D, KvFmt F, int STAGES, bool TR>
 struct DecodeSmem {
     static constexpr uint32_t kTileBytes = DecGeom<D, F>::kTileBytes;   // K or V of one stage
     static constexpr uint32_t kStageBytes = 2 * kTileBytes;
@@ -119,8 +117,12 @@ struct DecodeSmem {
     // After the ring has drained it is reused for the partial results:
     //   per-warp partials  part[WT][HS][D], pm[WT][HS], pl[WT][HS]
     //   per-CTA partial    co[HS][D], cm[HS], cl[HS]
-    static constexpr uint32_t kPartBytes = 4 * 16 * D * 4;            // WT * HS <= 64 rows
-    static_assert(kPartBytes * 2 + 4 * 64 * 4 <= kRingBytes, "partials must fit in the drained ring");
+    // (WT * HS <= 64 rows, HS <= 64; the transposed path has HS <= 8, WT = 4)
+    static constexpr uint32_t kPartRows = TR ? 32 : 64;
+    static constexpr uint32_t kCoRows = TR ? 8 : 64;
+    static constexpr uint32_t kPartBytes = kPartRows * D * 4;
+    static_assert(kPartBytes + 4 * 64 * 2 + kCoRows * D * 4 + 4 * 64 * 2 <= kRingBytes,
+                  "partials must fit in the drained ring");
 };
 
 // Consumer of a group of at most 8 query heads, with the products transposed so
@@ -140,7 +142,7 @@ __device__ __forceinline__ void consume_transposed(const DecodeParams &p, uint8_
                                                    int HS, int L, int first, int n_stages, float k_scale,
                                                    float (&o)[D / 8][4], float (&m_run)[2], float (&l_run)[2]) {
     using Geo = DecGeom<D, F>;
-    using SM = DecodeSmem<D, F, STAGES>;
+    using SM = DecodeSmem<D, F, STAGES, true>;
     constexpr bool FP8 = Geo::kFp8;
     constexpr int TOK = Geo::kTok;
     constexpr int RB = Geo::kRowBytes;
@@ -212,11 +214,11 @@ __device__ __forceinline__ void consume_transposed(const DecodeParams &p, uint8_
                     // x0: tokens 0-7 of k-step 2kp; x1: tokens 8-15; x2, x3: the same for k-step 2kp+1
                     uint32_t x0, x1, x2, x3;
                     ldmatrix_x4(x0, x1, x2, x3, rowaddr + (((2 * kp + achk) ^ sw) << 4));
-                    const uint32_t a0[4] = {e4m3x2_to_f16x2(x0), e4m3x2_to_f16x2(x1), e4m3x2_to_f16x2(x0 >> 16),
-                                            e4m3x2_to_f16x2(x1 >> 16)};
+                    const uint32_t a0[4] = {e4m3x2_to_f16x2_lo(x0), e4m3x2_to_f16x2_lo(x1), e4m3x2_to_f16x2_hi(x0),
+                                            e4m3x2_to_f16x2_hi(x1)};
                     mma_f16_16816(s[tt], a0, qb[2 * kp][0], qb[2 * kp][1]);
-                    const uint32_t a1[4] = {e4m3x2_to_f16x2(x2), e4m3x2_to_f16x2(x3), e4m3x2_to_f16x2(x2 >> 16),
-                                            e4m3x2_to_f16x2(x3 >> 16)};
+                    const uint32_t a1[4] = {e4m3x2_to_f16x2_lo(x2), e4m3x2_to_f16x2_lo(x3), e4m3x2_to_f16x2_hi(x2),
+                                            e4m3x2_to_f16x2_hi(x3)};
                     mma_f16_16816(s[tt], a1, qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
                 }
             }
@@ -285,10 +287,12 @@ __device__ __forceinline__ void consume_transposed(const DecodeParams &p, uint8_
         l_run[1] += ls.y;
         // O^T += V^T P^T.  On edge stages the V values of invalid rows are zeroed in
         // registers: each half of a transposed fragment register is one token.
+        auto pv = [&](auto masked) {
+          constexpr bool MASKED = decltype(masked)::value;
 #pragma unroll
-        for (int tt = 0; tt < TT; ++tt) {
+          for (int tt = 0; tt < TT; ++tt) {
             uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
-            if (partial) {
+            if constexpr (MASKED) {
                 const int row = tw0 + tt * 16 + 2 * q4;
                 auto ok = [&](int r) { return r >= row_lo && r < row_hi; };
                 mlo = (ok(row) ? 0x0000FFFFu : 0u) | (ok(row + 1) ? 0xFFFF0000u : 0u);
@@ -303,10 +307,12 @@ __device__ __forceinline__ void consume_transposed(const DecodeParams &p, uint8_
                     uint32_t a[4];
                     ldmatrix_x4_trans(a[0], a[1], a[2], a[3],
                                       rowaddr + (chunk >> 3) * Geo::kPanelBytes + (((chunk & 7) ^ (lane & 7)) << 4));
-                    a[0] &= mlo;
-                    a[1] &= mlo;
-                    a[2] &= mhi;
-                    a[3] &= mhi;
+                    if constexpr (MASKED) {
+                        a[0] &= mlo;
+                        a[1] &= mlo;
+                        a[2] &= mhi;
+                        a[3] &= mhi;
+                    }
                     mma_bf16_16816(o[mt], a, pb[tt][0], pb[tt][1]);
                 }
             } else {
@@ -317,19 +323,30 @@ __device__ __forceinline__ void consume_transposed(const DecodeParams &p, uint8_
                     // The permute puts the even channel's token pair in the low half, the odd's in the high.
                     uint32_t x0, x1, x2, x3;
                     ldmatrix_x4_trans(x0, x1, x2, x3, rowaddr + (((2 * cp + achk) ^ sw) << 4));
-                    x0 = __byte_perm(x0 & mlo, 0, 0x3120);
-                    x1 = __byte_perm(x1 & mhi, 0, 0x3120);
-                    x2 = __byte_perm(x2 & mlo, 0, 0x3120);
-                    x3 = __byte_perm(x3 & mhi, 0, 0x3120);
-                    const uint32_t a0[4] = {e4m3x2_to_f16x2(x0), e4m3x2_to_f16x2(x0 >> 16), e4m3x2_to_f16x2(x1),
-                                            e4m3x2_to_f16x2(x1 >> 16)};
+                    if constexpr (MASKED) {
+                        x0 &= mlo;
+                        x1 &= mhi;
+                        x2 &= mlo;
+                        x3 &= mhi;
+                    }
+                    x0 = __byte_perm(x0, 0, 0x3120);
+                    x1 = __byte_perm(x1, 0, 0x3120);
+                    x2 = __byte_perm(x2, 0, 0x3120);
+                    x3 = __byte_perm(x3, 0, 0x3120);
+                    const uint32_t a0[4] = {e4m3x2_to_f16x2_lo(x0), e4m3x2_to_f16x2_hi(x0), e4m3x2_to_f16x2_lo(x1),
+                                            e4m3x2_to_f16x2_hi(x1)};
                     mma_f16_16816(o[2 * cp], a0, pb[tt][0], pb[tt][1]);
-                    const uint32_t a1[4] = {e4m3x2_to_f16x2(x2), e4m3x2_to_f16x2(x2 >> 16), e4m3x2_to_f16x2(x3),
-                                            e4m3x2_to_f16x2(x3 >> 16)};
+                    const uint32_t a1[4] = {e4m3x2_to_f16x2_lo(x2), e4m3x2_to_f16x2_hi(x2), e4m3x2_to_f16x2_lo(x3),
+                                            e4m3x2_to_f16x2_hi(x3)};
                     mma_f16_16816(o[2 * cp + 1], a1, pb[tt][0], pb[tt][1]);
                 }
             }
-        }
+          }
+        };
+        if (partial)
+            pv(std::true_type{});
+        else
+            pv(std::false_type{});
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
     }
@@ -344,12 +361,12 @@ __device__ __forceinline__ void consume_transposed(const DecodeParams &p, uint8_
 // WT = token sub-ranges per stage (4, 2 or 1): consumer warp w serves m-tile
 // w / WT (16 query heads) on tokens [(w % WT) * TOK / WT, ...) of every stage,
 // in passes of at most 32 (d = 128) or 64 (d = 64) tokens.
-template <int D, int STAGES, int WT, KvFmt F, bool PAGED, bool TR>
-__global__ void __launch_bounds__(kDecThreads, 2)
+template <int D, int STAGES, int WT, KvFmt F, bool PAGED, bool TR, int MINB>
+__global__ void __launch_bounds__(kDecThreads, MINB)
     gqa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const DecodeParams p) {
     using Geo = DecGeom<D, F>;
-    using SM = DecodeSmem<D, F, STAGES>;
+    using SM = DecodeSmem<D, F, STAGES, TR>;
     constexpr bool FP8 = Geo::kFp8;
     constexpr int TOK = Geo::kTok;
     constexpr int RB = Geo::kRowBytes;
@@ -578,11 +595,11 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                             // x0: tokens 0-7, k-step 2kp; x1: tokens 8-15, 2kp; x2: 0-7, 2kp+1; x3: 8-15, 2kp+1
                             uint32_t x0, x1, x2, x3;
                             ldmatrix_x4(x0, x1, x2, x3, cbase + (np * 16 + frow) * RB);
-                            mma_f16_16816(s[2 * np], qa[2 * kp], e4m3x2_to_f16x2(x0), e4m3x2_to_f16x2(x0 >> 16));
-                            mma_f16_16816(s[2 * np + 1], qa[2 * kp], e4m3x2_to_f16x2(x1), e4m3x2_to_f16x2(x1 >> 16));
-                            mma_f16_16816(s[2 * np], qa[2 * kp + 1], e4m3x2_to_f16x2(x2), e4m3x2_to_f16x2(x2 >> 16));
-                            mma_f16_16816(s[2 * np + 1], qa[2 * kp + 1], e4m3x2_to_f16x2(x3),
-                                          e4m3x2_to_f16x2(x3 >> 16));
+                            mma_f16_16816(s[2 * np], qa[2 * kp], e4m3x2_to_f16x2_lo(x0), e4m3x2_to_f16x2_hi(x0));
+                            mma_f16_16816(s[2 * np + 1], qa[2 * kp], e4m3x2_to_f16x2_lo(x1), e4m3x2_to_f16x2_hi(x1));
+                            mma_f16_16816(s[2 * np], qa[2 * kp + 1], e4m3x2_to_f16x2_lo(x2), e4m3x2_to_f16x2_hi(x2));
+                            mma_f16_16816(s[2 * np + 1], qa[2 * kp + 1], e4m3x2_to_f16x2_lo(x3),
+                                          e4m3x2_to_f16x2_hi(x3));
                         }
                     }
                 }
@@ -657,10 +674,12 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                 l_run[1] += ls1.x + ls1.y;
                 // O += P V.  On edge passes the V values of invalid rows are zeroed in
                 // registers: each half of a transposed fragment register is one token.
+                auto pv = [&](auto masked) {
+                  constexpr bool MASKED = decltype(masked)::value;
 #pragma unroll
-                for (int kk = 0; kk < KKS; ++kk) {
+                  for (int kk = 0; kk < KKS; ++kk) {
                     uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
-                    if (partial) {
+                    if constexpr (MASKED) {
                         const int row = tw0 + kk * 16 + cq;   // this lane's tokens: row, row + 1 (and + 8)
                         auto ok = [&](int r) { return r >= row_lo && r < row_hi; };
                         mlo = (ok(row) ? 0x0000FFFFu : 0u) | (ok(row + 1) ? 0xFFFF0000u : 0u);
@@ -675,8 +694,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                             ldmatrix_x4_trans(b0, b1, b2, b3,
                                               rowaddr + (chunk >> 3) * Geo::kPanelBytes +
                                                   (((chunk & 7) ^ (lane & 7)) << 4));
-                            mma_bf16_16816(o[2 * dp], pa[kk], b0 & mlo, b1 & mhi);
-                            mma_bf16_16816(o[2 * dp + 1], pa[kk], b2 & mlo, b3 & mhi);
+                            if constexpr (MASKED) {
+                                b0 &= mlo;
+                                b1 &= mhi;
+                                b2 &= mlo;
+                                b3 &= mhi;
+                            }
+                            mma_bf16_16816(o[2 * dp], pa[kk], b0, b1);
+                            mma_bf16_16816(o[2 * dp + 1], pa[kk], b2, b3);
                         }
                     } else {
 #pragma unroll
@@ -686,17 +711,28 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                             // the permute makes the low half the even channel's pair and the high half the odd's.
                             uint32_t x0, x1, x2, x3;
                             ldmatrix_x4_trans(x0, x1, x2, x3, rowaddr + (((2 * cp + fchk) ^ sw) << 4));
-                            x0 = __byte_perm(x0 & mlo, 0, 0x3120);
-                            x1 = __byte_perm(x1 & mhi, 0, 0x3120);
-                            x2 = __byte_perm(x2 & mlo, 0, 0x3120);
-                            x3 = __byte_perm(x3 & mhi, 0, 0x3120);
-                            mma_f16_16816(o[4 * cp + 0], pa[kk], e4m3x2_to_f16x2(x0), e4m3x2_to_f16x2(x1));
-                            mma_f16_16816(o[4 * cp + 1], pa[kk], e4m3x2_to_f16x2(x0 >> 16), e4m3x2_to_f16x2(x1 >> 16));
-                            mma_f16_16816(o[4 * cp + 2], pa[kk], e4m3x2_to_f16x2(x2), e4m3x2_to_f16x2(x3));
-                            mma_f16_16816(o[4 * cp + 3], pa[kk], e4m3x2_to_f16x2(x2 >> 16), e4m3x2_to_f16x2(x3 >> 16));
+                            if constexpr (MASKED) {
+                                x0 &= mlo;
+                                x1 &= mhi;
+                                x2 &= mlo;
+                                x3 &= mhi;
+                            }
+                            x0 = __byte_perm(x0, 0, 0x3120);
+                            x1 = __byte_perm(x1, 0, 0x3120);
+                            x2 = __byte_perm(x2, 0, 0x3120);
+                            x3 = __byte_perm(x3, 0, 0x3120);
+                            mma_f16_16816(o[4 * cp + 0], pa[kk], e4m3x2_to_f16x2_lo(x0), e4m3x2_to_f16x2_lo(x1));
+                            mma_f16_16816(o[4 * cp + 1], pa[kk], e4m3x2_to_f16x2_hi(x0), e4m3x2_to_f16x2_hi(x1));
+                            mma_f16_16816(o[4 * cp + 2], pa[kk], e4m3x2_to_f16x2_lo(x2), e4m3x2_to_f16x2_lo(x3));
+                            mma_f16_16816(o[4 * cp + 3], pa[kk], e4m3x2_to_f16x2_hi(x2), e4m3x2_to_f16x2_hi(x3));
                         }
                     }
-                }
+                  }
+                };
+                if (partial)
+                    pv(std::true_type{});
+                else
+                    pv(std::false_type{});
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
@@ -711,10 +747,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     // ---------------------------------------------------------------- combine
     __syncthreads();   // the ring has drained: reuse it for the partials
     float *part = reinterpret_cast<float *>(smem);               // [WT][HS][D]
-    float *pm = part + 4 * 16 * D;                               // [WT][HS]
+    float *pm = part + SM::kPartRows * D;                        // [WT][HS]
     float *pl = pm + 64;                                         // [WT][HS]
     float *co = reinterpret_cast<float *>(smem + SM::kPartBytes + 4 * 64 * 2);   // [HS][D]
-    float *cm = co + 64 * D;                                     // [HS]
+    float *cm = co + SM::kCoRows * D;                            // [HS]
     float *cl = cm + 64;                                         // [HS]
     if (consumer && TR) {
         // O^T m-tile mt: rows = channels, columns = heads 2j, 2j+1 (j = lane % 4)
@@ -831,11 +867,11 @@ struct DecodeCall {
     cudaStream_t stream;
 };
 
-template <int D, int STAGES, int WT, KvFmt F, bool PAGED, bool TR>
+template <int D, int STAGES, int WT, KvFmt F, bool PAGED, bool TR, int MINB = 2>
 static int launch_decode_t(const DecodeCall &c) {
     using Geo = DecGeom<D, F>;
-    using SM = DecodeSmem<D, F, STAGES>;
-    auto kern = gqa_decode_kernel<D, STAGES, WT, F, PAGED, TR>;
+    using SM = DecodeSmem<D, F, STAGES, TR>;
+    auto kern = gqa_decode_kernel<D, STAGES, WT, F, PAGED, TR, MINB>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 3;
     static unsigned long long attr_done = 0;   // one bit per device
@@ -877,7 +913,8 @@ static int launch_decode_t(const DecodeCall &c) {
     // Splits per (sequence, KV head): as many as fit in one wave of resident
     // CTAs (two per SM), at most the cluster limit.  Longer CTAs amortise their
     // start and merge; a second, partial wave would leave SMs idle at the end.
-    const long slots = static_cast<long>(GQA_DECODE_CTAS_PER_SM) * sms;
+    // (MINB resident CTAs per SM: 2 with a 3-stage ring, 3 with a 2-stage ring.)
+    const long slots = static_cast<long>(MINB) * sms;
     const int P = static_cast<int>(std::max(1L, std::min(static_cast<long>(GQA_DECODE_MAX_SPLIT), slots / units)));
 
     DecodeParams prm;
@@ -924,6 +961,7 @@ static int launch_decode_d(const DecodeCall &c) {
     return launch_decode_t<D, STAGES, 1, F, PAGED, false>(c);
 }
 
+// Ring depth: 96 KB of stages per CTA, two CTAs per SM.
 template <KvFmt F, bool PAGED>
 static int launch_decode_f(const DecodeCall &c, int d) {
     if (d == 128) return launch_decode_d<128, 3, F, PAGED>(c);

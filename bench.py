@@ -8,7 +8,9 @@ each), inputs resident in device memory; three copies of the KV cache are
 rotated so every step reads a cache L2 has not seen for two steps (each copy,
 256 MiB, is twice the 126 MB L2).  The causal prefill workload (B=4,
 S=4096, h=32, n_kv=8, d=128) is timed in the same run and reported under
-"prefill".  Under torchrun every rank runs the same per-GPU workload (the
+"prefill", and the same decode workload over an E4M3 cache, a paged bf16
+cache and a paged E4M3 cache under "decode_fp8", "decode_paged" and
+"decode_paged_fp8".  Under torchrun every rank runs the same per-GPU workload (the
 (sequence, KV head) units are independent: weak scaling, no collective on the
 data path); the time is the max over ranks.
 """
@@ -230,6 +232,51 @@ def decode_leg(args, device, world, clocks):
     return res
 
 
+def cache_variant_leg(kind, args, device, world, page_size=64):
+    """The GQA decode workload over another cache: "fp8" (packed E4M3, one scale
+    per KV head), "paged" (bf16, pages of `page_size` tokens in a seeded random
+    order) or "paged_fp8".  Copies rotated so each step reads a cache L2 has not
+    seen for two steps; CUDA-event time per launch."""
+    import torch
+    import attention_gqa_decode_b200 as gqa
+    from attention_gqa_decode_b200 import inputs, metrics
+    w = inputs.GQA_DECODE_70B
+    fp8 = kind.endswith("fp8")
+    if fp8:
+        q, k, v, ksc, vsc, lens = inputs.decode_fp8_inputs(w.seed, w.B, w.h, w.n_kv, w.d, w.kv_len)
+        ksc, vsc = ksc.to(device), vsc.to(device)
+    else:
+        q, k, v, lens = inputs.workload_inputs(w)
+        ksc = vsc = None
+    bt = None
+    if kind.startswith("paged"):
+        k, v, bt = inputs.page_caches(w.seed, k, v, lens, page_size)
+        bt = bt.to(device)
+    kv_bytes = metrics.decode_kv_bytes(lens.tolist(), w.n_kv, w.d) // (2 if fp8 else 1)
+    copies = max(3, -(-3 * 128 * 1024 * 1024 // kv_bytes))   # every copy set is >= 3 x 128 MiB
+    qd, ld = q.to(device), lens.to(device)
+    ks = [k.to(device) for _ in range(copies)]
+    vs = [v.to(device) for _ in range(copies)]
+    out = torch.empty_like(qd)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i):
+        c = i % copies
+        if bt is not None:
+            gqa.decode_paged(qd, ks[c], vs[c], bt, ld, k_scale=ksc, v_scale=vsc, out=out)
+        else:
+            gqa.decode_fp8(qd, ks[c], vs[c], ksc, vsc, ld, out=out)
+
+    steps = max(3, min(args.steps, 300))
+    barrier(world)
+    per, _ = time_launches(step, steps, max(3, args.warmup), stream)
+    barrier(world)
+    kern_ms = multirank.max_over_ranks(statistics.mean(per), device)
+    if gqa.gqa_get_device_status() != 0:
+        raise RuntimeError(f"device status after the {kind} decode leg")
+    return {"kv_bytes": kv_bytes, "kernel_ms": kern_ms, "steps": steps, "copies": copies}
+
+
 def prefill_leg(args, device, world):
     import torch
     import attention_gqa_decode_b200 as gqa
@@ -265,6 +312,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true", help="skip the E4M3 / paged cache legs")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local = dist_env()
@@ -299,6 +347,11 @@ def main():
     clocks = ClockSampler(device)
     dec = decode_leg(args, device, world, clocks)
     pre = None if args.no_prefill else prefill_leg(args, device, world)
+    variants = {} if args.no_variants else {
+        "decode_fp8": cache_variant_leg("fp8", args, device, world),
+        "decode_paged": cache_variant_leg("paged", args, device, world),
+        "decode_paged_fp8": cache_variant_leg("paged_fp8", args, device, world),
+    }
 
     value = multirank.job_throughput(dec["kv_bytes"] * args.steps, dec["total_ms"], device) / 1e9
     achieved = dec["kv_bytes"] / (dec["kernel_ms"] / 1e3) / 1e9
@@ -324,6 +377,19 @@ def main():
                          "frac": tf / pk["bf16"], "frac_of_sustained": tf / pk["bf16_sustained"],
                          "traffic": kernel_traffic("gqa_prefill_kernel"),
                          "algorithmic_flops_per_launch": pre["flops"], "peak_source": pk["src"]}}
+    desc = {"decode_fp8": ("E4M3 cache, one fp32 scale per KV head", "gqa_decode_kernel[e4m3]"),
+            "decode_paged": ("bf16 cache in 64-token pages, seeded random page order", "gqa_decode_kernel[paged]"),
+            "decode_paged_fp8": ("E4M3 cache in 64-token pages", "gqa_decode_kernel[paged,e4m3]")}
+    for name, r in variants.items():
+        gbs = r["kv_bytes"] / (r["kernel_ms"] / 1e3) / 1e9
+        line[name] = {
+            "metric": "GQA decode KV GB/s", "workload": f"{w.name}, {desc[name][0]}",
+            "value": world * gbs, "unit": "GB/s", "ms_per_call": r["kernel_ms"], "steps": r["steps"],
+            "tokens_per_s": world * w.B / (r["kernel_ms"] / 1e3),
+            "l2": f"{r['copies']} cache copies rotated",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm"], "traffic": kernel_traffic(desc[name][1]),
+                         "algorithmic_bytes_per_launch": r["kv_bytes"], "peak_source": pk["src"]}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_decode_leg(target_s=10.0)
     if world > 1:
