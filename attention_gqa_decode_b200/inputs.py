@@ -156,17 +156,19 @@ def decode_fp8_inputs(seed: int, B: int, h: int, n_kv: int, d: int, seqlens):
     return q, kc, vc, ks, vs, seqlens
 
 
-def page_caches(seed: int, k: torch.Tensor, v: torch.Tensor, seqlens, page_size: int, spare_pages: int = 0):
+def page_caches(seed: int, k: torch.Tensor, v: torch.Tensor, seqlens, page_size: int, spare_pages: int = 0,
+                reserve: int = 0):
     """Cut packed caches [sum(seqlens), n_kv, d] into pages.
 
     Returns (k_pages, v_pages [num_pages, page_size, n_kv, d], block_table
     int32 [B, max_blocks]).  Pages are placed in a seeded random order;
     block-table entries past a sequence's last page are -1; unused slots and
-    the ``spare_pages`` extra pages hold NaN.
+    the ``spare_pages`` extra pages hold NaN.  ``reserve`` extra tokens per
+    sequence get pages too (left NaN), for a chunk to be appended.
     """
     lens = torch.as_tensor(seqlens, dtype=torch.int32).reshape(-1)
     B = lens.numel()
-    n_blocks = [(max(int(L), 0) + page_size - 1) // page_size for L in lens.tolist()]
+    n_blocks = [(max(int(L), 0) + reserve + page_size - 1) // page_size for L in lens.tolist()]
     max_blocks = max(1, max(n_blocks) if n_blocks else 1)
     num_pages = sum(n_blocks) + spare_pages
     g = _gen(seed)
@@ -185,9 +187,30 @@ def page_caches(seed: int, k: torch.Tensor, v: torch.Tensor, seqlens, page_size:
         for j in range(n_blocks[b]):
             page = int(order[used])
             used += 1
-            n = min(page_size, L - j * page_size)
+            n = max(0, min(page_size, L - j * page_size))
             kp[page, :n] = kr[row + j * page_size: row + j * page_size + n]
             vp[page, :n] = vr[row + j * page_size: row + j * page_size + n]
             bt[b, j] = page
         row += L
     return kp.view(k.dtype)[:num_pages], vp.view(v.dtype)[:num_pages], bt
+
+
+def chunk_prefill_inputs(seed: int, B: int, S_q: int, past_lens, h: int, n_kv: int, d: int, page_size: int,
+                         spare_pages: int = 0):
+    """A chunk of S_q new tokens per sequence after past_lens[b] cached ones.
+
+    Returns q [B,S_q,h,d], k_new and v_new [B,S_q,n_kv,d] (bf16), the paged
+    caches holding the past tokens with pages reserved for the chunk (NaN
+    until written), the block table, and past_lens int32 [B].  The past rows
+    are drawn first (as a packed decode cache), then q, k_new, v_new.
+    """
+    past = torch.as_tensor(past_lens, dtype=torch.int32).reshape(B)
+    g = _gen(seed)
+    total = int(past.clamp(min=0).sum())
+    k_past = _randn_bf16(g, (total, n_kv, d))
+    v_past = _randn_bf16(g, (total, n_kv, d))
+    q = _randn_bf16(g, (B, S_q, h, d))
+    k_new = _randn_bf16(g, (B, S_q, n_kv, d))
+    v_new = _randn_bf16(g, (B, S_q, n_kv, d))
+    kp, vp, bt = page_caches(seed + 1, k_past, v_past, past, page_size, spare_pages=spare_pages, reserve=S_q)
+    return q, k_new, v_new, kp, vp, bt, past

@@ -61,6 +61,9 @@ def _load():
             lib.oracle_decode_general.argtypes = ([_u16p, ctypes.c_void_p, ctypes.c_void_p, _int, _f32p, _f32p,
                                                    _i32p, _i32p, _int, _int, _int, _f64p] + [_int] * 4 +
                                                   [ctypes.c_double, _int])
+            lib.oracle_prefill_paged.argtypes = ([_u16p, _u16p, _u16p, _u16p, _u16p, _i32p, _int, _int, _int, _i32p,
+                                                  _f64p] + [_int] * 5 + [ctypes.c_double, _int])
+            lib.oracle_prefill_paged.restype = _int
             lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
             lib.oracle_e4m3_value.restype = ctypes.c_double
             for f in (lib.oracle_prefill, lib.oracle_prefill_rows, lib.oracle_decode, lib.oracle_prefill_probs,
@@ -217,3 +220,29 @@ def decode_general(q, k_cache, v_cache, seqlens, *, fp8: bool = False, k_scale=N
     if rc:
         raise ValueError("oracle_decode_general rejected its arguments")
     return out
+
+
+def prefill_paged(q, k_new, v_new, k_pages, v_pages, block_table, past_lens, scale: float | None = None):
+    """Chunked causal prefill over a paged bf16 cache, with the append.
+
+    q [B,S_q,h,d], k_new/v_new [B,S_q,n_kv,d], pages [num_pages,page_size,n_kv,d],
+    block_table [B,max_blocks], past_lens [B].  Returns (out fp64 [B,S_q,h,d],
+    k_pages_after, v_pages_after) -- the pages after the chunk's K/V were written
+    at positions past_lens[b] .. past_lens[b] + S_q - 1 (as uint16 bf16 bits).
+    """
+    qb, kn, vn = _bits(q), _bits(k_new), _bits(v_new)
+    kp, vp = _bits(k_pages).copy(), _bits(v_pages).copy()
+    B, S_q, h, d = qb.shape
+    n_kv = kn.shape[2]
+    num_pages, page_size = kp.shape[0], kp.shape[1]
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32).reshape(B, -1))
+    past = np.ascontiguousarray(np.asarray(past_lens, dtype=np.int32).reshape(B))
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.empty((B, S_q, h, d), dtype=np.float64)
+    rc = _load().oracle_prefill_paged(_p(qb, _u16p), _p(kn, _u16p), _p(vn, _u16p), _p(kp, _u16p), _p(vp, _u16p),
+                                      _p(bt, _i32p), bt.shape[1], page_size, num_pages, _p(past, _i32p),
+                                      _p(out, _f64p), B, S_q, h, n_kv, d, float(scale), 0)
+    if rc:
+        raise ValueError("oracle_prefill_paged rejected its arguments")
+    return out, kp, vp

@@ -409,3 +409,78 @@ int oracle_decode_general(const uint16_t *q, const void *k_cache, const void *v_
     free(off);
     return rc;
 }
+
+/* Chunked prefill over a paged bf16 cache, with the cache write.
+ *   Same pages as oracle_decode_general: [num_pages, page_size, n_kv, d], token
+ *   t of sequence b in slot t % page_size of page block_table[b][t / page_size].
+ *   Sequence b holds past_lens[b] cached tokens; the chunk adds S_q tokens:
+ *   q [B, S_q, h, d], k_new / v_new [B, S_q, n_kv, d].
+ * Step 1 (the append; "Evolution of AI Attention Mechanisms", "MHA
+ * Implementation": new K/V are concatenated after the past ones): row t of
+ * k_new[b] / v_new[b] is copied to cache position past_lens[b] + t, for every
+ * KV head.  k_pages / v_pages are updated in place.
+ * Step 2: query row r of sequence b sits at position past_lens[b] + r and sees
+ * keys at positions <= past_lens[b] + r (bottom-right causal), read back from
+ * the updated pages.  out [B, S_q, h, d] fp64.
+ * Returns -1 for bad shapes, a negative past length, a length past the block
+ * table, or a page id outside [0, num_pages). */
+int oracle_prefill_paged(const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new,
+                         uint16_t *k_pages, uint16_t *v_pages, const int32_t *block_table, int max_blocks,
+                         int page_size, int num_pages, const int32_t *past_lens, double *out,
+                         int B, int S_q, int h, int n_kv, int d, double scale, int n_threads) {
+    (void)n_threads;
+    if (!check_shape(B, h, n_kv, d) || S_q <= 0 || max_blocks <= 0 || page_size <= 0 || num_pages <= 0) return -1;
+    for (int b = 0; b < B; ++b) {
+        long total = (long)past_lens[b] + S_q;
+        if (past_lens[b] < 0 || total > (long)max_blocks * page_size) return -1;
+        for (long t = 0; t < total; t += page_size) {
+            int page = block_table[(size_t)b * max_blocks + t / page_size];
+            if (page < 0 || page >= num_pages) return -1;
+        }
+    }
+    const size_t row = (size_t)n_kv * d;   /* elements of one cached token */
+    /* step 1: the append */
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < S_q; ++t) {
+            long pos = (long)past_lens[b] + t;
+            int page = block_table[(size_t)b * max_blocks + pos / page_size];
+            size_t dst = ((size_t)page * page_size + (size_t)(pos % page_size)) * row;
+            size_t src = ((size_t)b * S_q + t) * row;
+            memcpy(k_pages + dst, k_new + src, sizeof(uint16_t) * row);
+            memcpy(v_pages + dst, v_new + src, sizeof(uint16_t) * row);
+        }
+    /* step 2: attention over the gathered cache */
+    int G = h / n_kv;
+    for (int b = 0; b < B; ++b) {
+        int total = past_lens[b] + S_q;
+        double *kd = (double *)malloc(sizeof(double) * (size_t)total * d);
+        double *vd = (double *)malloc(sizeof(double) * (size_t)total * d);
+        double *qd = (double *)malloc(sizeof(double) * (size_t)S_q * d);
+        double *o = (double *)malloc(sizeof(double) * (size_t)S_q * d);
+        int *vis = (int *)malloc(sizeof(int) * (size_t)S_q);
+        if (!kd || !vd || !qd || !o || !vis) { free(kd); free(vd); free(qd); free(o); free(vis); return -1; }
+        for (int r = 0; r < S_q; ++r) vis[r] = past_lens[b] + r + 1;
+        for (int g = 0; g < n_kv; ++g) {
+            for (int t = 0; t < total; ++t) {
+                int page = block_table[(size_t)b * max_blocks + t / page_size];
+                size_t base = ((size_t)page * page_size + (size_t)(t % page_size)) * row + (size_t)g * d;
+                for (int c = 0; c < d; ++c) {
+                    kd[(size_t)t * d + c] = bf16_value(k_pages[base + c]);
+                    vd[(size_t)t * d + c] = bf16_value(v_pages[base + c]);
+                }
+            }
+            for (int i = g * G; i < (g + 1) * G; ++i) {
+                for (int r = 0; r < S_q; ++r)
+                    for (int c = 0; c < d; ++c)
+                        qd[(size_t)r * d + c] = bf16_value(q[(((size_t)b * S_q + r) * h + i) * d + c]);
+                if (attend_f64(qd, S_q, kd, vd, total, d, vis, scale, o, NULL)) {
+                    free(kd); free(vd); free(qd); free(o); free(vis); return -1;
+                }
+                for (int r = 0; r < S_q; ++r)
+                    memcpy(out + (((size_t)b * S_q + r) * h + i) * d, o + (size_t)r * d, sizeof(double) * (size_t)d);
+            }
+        }
+        free(kd); free(vd); free(qd); free(o); free(vis);
+    }
+    return 0;
+}
