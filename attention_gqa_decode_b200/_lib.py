@@ -21,6 +21,7 @@ SIGNATURES = {
     "gqa_decode_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_paged": ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_paged_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
+    "gqa_prefill_paged": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_status_string": ([_i], ctypes.c_char_p),
     "gqa_get_device_status": ([_vp], _i),
 }
@@ -88,6 +89,12 @@ def gqa_decode_paged_fp8(q, k_pages, v_pages, k_scale, v_scale, block_table, max
                          seqlens, out, B, h, n_kv, d_h, scale, stream) -> int:
     return lib().gqa_decode_paged_fp8(q, k_pages, v_pages, k_scale, v_scale, block_table, max_blocks, page_size,
                                       num_pages, seqlens, out, B, h, n_kv, d_h, float(scale), stream)
+
+
+def gqa_prefill_paged(q, k_new, v_new, k_pages, v_pages, block_table, max_blocks, page_size, num_pages, past_lens,
+                      out, B, S_q, h, n_kv, d_h, scale, stream) -> int:
+    return lib().gqa_prefill_paged(q, k_new, v_new, k_pages, v_pages, block_table, max_blocks, page_size, num_pages,
+                                   past_lens, out, B, S_q, h, n_kv, d_h, float(scale), stream)
 
 
 def gqa_get_device_status(stream=None) -> int:
@@ -277,4 +284,45 @@ def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale: float | None 
                                   _stream_ptr(stream))
     if st != GQA_OK:
         raise GQAError(st, "gqa_decode_paged_fp8" if fp8 else "gqa_decode_paged")
+    return out
+
+
+def prefill_paged(q, k_new, v_new, k_pages, v_pages, block_table, past_lens, scale: float | None = None, out=None,
+                  stream=None):
+    """Chunked causal prefill over a paged bf16 cache, appending the chunk.
+
+    q [B,S_q,h,d], k_new/v_new [B,S_q,n_kv,d], pages [num_pages,page_size,n_kv,d]
+    (written in place at positions past_lens[b] .. past_lens[b]+S_q-1),
+    block_table int32 [B,max_blocks], past_lens int32 [B] (CUDA).  Query row r
+    attends to keys at positions <= past_lens[b] + r.  Returns out [B,S_q,h,d].
+    """
+    import torch
+    _check(q, "q", 4), _check(k_new, "k_new", 4), _check(v_new, "v_new", 4)
+    _check(k_pages, "k_pages", 4), _check(v_pages, "v_pages", 4)
+    B, S_q, h, d = q.shape
+    if tuple(k_new.shape) != tuple(v_new.shape) or k_new.shape[0] != B or k_new.shape[1] != S_q \
+            or k_new.shape[3] != d:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k_new{tuple(k_new.shape)} v_new{tuple(v_new.shape)}")
+    n_kv = k_new.shape[2]
+    num_pages, page_size, n_kv_p, d_p = k_pages.shape
+    if tuple(v_pages.shape) != tuple(k_pages.shape) or n_kv_p != n_kv or d_p != d:
+        raise ValueError(f"page shape mismatch {tuple(k_pages.shape)} {tuple(v_pages.shape)}")
+    if not isinstance(block_table, torch.Tensor) or block_table.dtype != torch.int32 or not block_table.is_cuda \
+            or block_table.dim() != 2 or block_table.shape[0] != B or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous int32 CUDA tensor [B, max_blocks]")
+    _check_seqlens(past_lens, B)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check(out, "out", 4)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    with torch.cuda.device(q.device):
+        st = gqa_prefill_paged(q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_pages.data_ptr(),
+                               v_pages.data_ptr(), block_table.data_ptr(), block_table.shape[1], page_size, num_pages,
+                               past_lens.data_ptr(), out.data_ptr(), B, S_q, h, n_kv, d, scale, _stream_ptr(stream))
+    if st != GQA_OK:
+        raise GQAError(st, "gqa_prefill_paged")
     return out

@@ -14,6 +14,10 @@ int launch_prefill(const void *q, const void *k, const void *v, void *out, int B
                    int d, int causal, float scale, cudaStream_t stream);
 int launch_decode(const void *q, const void *k, const void *v, const int32_t *seqlens, void *out, int B, int h,
                   int n_kv, int d, float scale, cudaStream_t stream);
+int launch_prefill_paged(const void *q, const void *k_new, const void *v_new, void *k_pages, void *v_pages,
+                         const int32_t *block_table, int max_blocks, int page_size, int num_pages,
+                         const int32_t *past_lens, void *out, int B, int S_q, int h, int n_kv, int d, float scale,
+                         cudaStream_t stream);
 int launch_decode_ex(const void *q, const void *k, const void *v, const float *k_scale, const float *v_scale,
                      const int32_t *seqlens, const int32_t *block_table, int max_blocks, int page_size,
                      int num_pages, void *out, int B, int h, int n_kv, int d, float scale, cudaStream_t stream);
@@ -178,6 +182,25 @@ int gqa_decode_paged_fp8(const void *q, const void *k_pages, const void *v_pages
     if (st != GQA_OK) return st;
     return gqa::launch_decode_ex(q, k_pages, v_pages, k_scale, v_scale, seqlens, block_table, max_blocks, page_size,
                                  num_pages, out, B, h, n_kv, d_h, scale, stream);
+}
+
+int gqa_prefill_paged(const void *q, const void *k_new, const void *v_new, void *k_pages, void *v_pages,
+                      const int32_t *block_table, int max_blocks, int page_size, int num_pages,
+                      const int32_t *past_lens, void *out, int B, int S_q, int h, int n_kv, int d_h, float scale,
+                      cudaStream_t stream) {
+    if (!q || !k_new || !v_new || !out || !past_lens) return GQA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(past_lens) & 3u))
+        return GQA_ERR_INVALID_ARG;
+    int st = caches_ok(k_pages, v_pages);
+    if (st == GQA_OK) st = pages_ok(block_table, max_blocks, page_size, num_pages);
+    if (st != GQA_OK) return st;
+    if (B <= 0 || S_q <= 0 || h <= 0 || n_kv <= 0 || h % n_kv != 0) return GQA_ERR_INVALID_ARG;
+    if (static_cast<long long>(S_q) > static_cast<long long>(max_blocks) * page_size) return GQA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return GQA_ERR_INVALID_ARG;
+    if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
+    return gqa::launch_prefill_paged(q, k_new, v_new, k_pages, v_pages, block_table, max_blocks, page_size,
+                                     num_pages, past_lens, out, B, S_q, h, n_kv, d_h, scale, stream);
 }
 
 const char *gqa_status_string(int status) {

@@ -27,6 +27,24 @@
 // The two query tiles ping-pong: while one warpgroup computes its softmax,
 // the tensor cores run the other tile's P V and next Q K^T.  Causal CTAs are
 // ordered heaviest first; tiles wholly above the diagonal are never loaded.
+//
+// Chunked prefill over a paged cache (PAGED): sequence b holds past_lens[b]
+// tokens in cache pages ("Multi-Query Attention (MQA)" (inferensys glossary),
+// "PagedAttention") and the call adds a chunk of S_q tokens whose K/V are
+// concatenated after them ("MHA Implementation", past_kv), so query row r
+// sees keys at positions <= past + r.  The key tiles are the past tiles,
+// loaded from the pages with one TMA box per page piece (page ids read one
+// tile ahead by the producer warp), then the chunk's tiles, loaded from the
+// new K/V directly.  The last past tile ends at position `past`: its columns
+// beyond are masked in the softmax, and its V rows beyond are zeroed in
+// shared memory by the MMA warp before the P V that reads them (whatever the
+// cache holds there, 0 * NaN must not reach O).  The append itself is done by
+// the two idle warps: the CTA of the first query head of a KV group copies
+// the new K/V rows of its own two query tiles into the pages, while the other
+// warps attend.  The attention never reads a slot that is being written:
+// past tiles only cover positions < past.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace gqa {
@@ -48,6 +66,11 @@ struct PrefillParams {
     int B, S_q, S_kv, h, n_kv, G, n_pairs, causal;
     float scale_log2;
     int *status;                   // the library's device status word
+    // chunked prefill over a paged cache
+    const int32_t *block_table, *past_lens;
+    const __nv_bfloat16 *k_new, *v_new;
+    __nv_bfloat16 *k_pages, *v_pages;
+    int max_blocks, page_size, num_pages;
 };
 
 template <int D>
@@ -67,10 +90,18 @@ __device__ __forceinline__ int kv_tiles_for(int rows_begin, int S_q, int S_kv, i
     return limit / kPfKeys + 1;
 }
 
-template <int D>
+// Key tiles a paged-chunk query tile starting at row rows_begin walks: all
+// past tiles, then the chunk's tiles up to its last row (causal).
+__device__ __forceinline__ int chunk_tiles_for(int rows_begin, int S_q, int n_past) {
+    if (rows_begin >= S_q) return 0;
+    return n_past + min(rows_begin + kPfRows - 1, S_q - 1) / kPfKeys + 1;
+}
+
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(kPfThreads, 1)
     gqa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
+                       const __grid_constant__ CUtensorMap tm_vp, const PrefillParams p) {
     using SM = PrefillSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -96,8 +127,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int pair = p.causal ? (p.n_pairs - 1 - pr) : pr;
     const int b = bh / p.h, head = bh % p.h, kvh = head / p.G;
     const int q0 = pair * 2 * kPfRows;
-    const int n_t0 = kv_tiles_for(q0, p.S_q, p.S_kv, p.causal);
-    const int n_t1 = kv_tiles_for(q0 + kPfRows, p.S_q, p.S_kv, p.causal);
+    // paged chunk: past tokens of this sequence (cut to what the block table can hold)
+    int past = 0;
+    if constexpr (PAGED) {
+        past = max(p.past_lens[b], 0);
+        const int cap = p.max_blocks * p.page_size - p.S_q;
+        if (past > cap) {
+            if (threadIdx.x == 0) record_status(p.status, kStatusInvalid);
+            past = max(cap, 0);
+        }
+    }
+    const int n_past = (past + kPfKeys - 1) / kPfKeys;
+    const int n_t0 = PAGED ? chunk_tiles_for(q0, p.S_q, n_past) : kv_tiles_for(q0, p.S_q, p.S_kv, p.causal);
+    const int n_t1 = PAGED ? chunk_tiles_for(q0 + kPfRows, p.S_q, n_past)
+                           : kv_tiles_for(q0 + kPfRows, p.S_q, p.S_kv, p.causal);
     const int nmax = max(n_t0, n_t1);
 
     if (threadIdx.x == 0) {
@@ -128,32 +171,77 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         regs_dec<kRegsOther>();   // warpgroup 2: producer, MMA issuer, two idle warps
         if (warp == 8) {
             // ------------------------------------------------------------ producer
+            // (the whole warp runs the loop; lane 0 waits and issues, lanes hold page ids)
             if (lane == 0) {
                 tma_prefetch_desc(&tm_q);
                 tma_prefetch_desc(&tm_k);
                 tma_prefetch_desc(&tm_v);
+                if (PAGED) {
+                    tma_prefetch_desc(&tm_kp);
+                    tma_prefetch_desc(&tm_vp);
+                }
                 mbar_arrive_expect_tx(qfull, SM::kQ);
                 for (int t = 0; t < 2; ++t)
                     for (int hf = 0; hf < D / 64; ++hf)
                         tma_load_4d(sQ + t * SM::kTile + hf * SM::kHalf, &tm_q, qfull, hf * 64, head, q0 + t * kPfRows, b);
-                int item = 0;
-                bool stop = false;
-                for (int j = 0; j < nmax && !stop; ++j) {
-                    for (int kv = 0; kv < 2; ++kv, ++item) {
-                        const int slot = item % kPfRing, use = item / kPfRing;
-                        if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, abort_flag, p.status)) { stop = true; break; }
+            }
+            const int pb = PAGED ? min(p.page_size, kPfKeys) : kPfKeys;   // rows per page box
+            // lane k: page id of piece k of past tile j (0 where there is none)
+            auto page_of = [&](int j) -> int {
+                int page = 0;
+                const int pos = j * kPfKeys + lane * pb;
+                if (PAGED && j < n_past && lane * pb < kPfKeys && pos < past) {
+                    page = p.block_table[static_cast<size_t>(b) * p.max_blocks + pos / p.page_size];
+                    if (page < 0 || page >= p.num_pages) {   // read as zeros, reported
+                        record_status(p.status, kStatusInvalid);
+                        page = p.num_pages;
+                    }
+                }
+                return page;
+            };
+            int next_pages = page_of(0);
+            int item = 0;
+            bool stop = false;
+            for (int j = 0; j < nmax && !stop; ++j) {
+                const int pages = next_pages;
+                if (PAGED && j + 1 < nmax) next_pages = page_of(j + 1);
+                for (int kv = 0; kv < 2; ++kv, ++item) {
+                    const int slot = item % kPfRing, use = item / kPfRing;
+                    int ok = 1;
+                    if (lane == 0 && use > 0) ok = mbar_wait(&empty[slot], (use - 1) & 1, abort_flag, p.status);
+                    if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                        stop = true;
+                        break;
+                    }
+                    uint8_t *dst = sRing + slot * SM::kTile;
+                    if (PAGED && j < n_past) {
+                        // rows [0, valid) of this tile are cached tokens: one box per page piece
+                        const int valid = min(kPfKeys, past - j * kPfKeys);
+                        const int nb = (valid + pb - 1) / pb;
+                        const CUtensorMap *map = kv ? &tm_vp : &tm_kp;
+                        if (lane == 0) mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nb * pb * 128 * (D / 64)));
+                        for (int k = 0; k < nb; ++k) {
+                            const int page = __shfl_sync(0xffffffffu, pages, k);
+                            if (lane == 0) {
+                                const int slot_in_page = (j * kPfKeys + k * pb) % p.page_size;
+                                for (int hf = 0; hf < D / 64; ++hf)
+                                    tma_load_4d(dst + hf * SM::kHalf + k * pb * 128, map, &full[slot], hf * 64, kvh,
+                                                slot_in_page, page);
+                            }
+                        }
+                    } else if (lane == 0) {
+                        // the chunk's own K/V (PAGED), or the K/V tensors
                         mbar_arrive_expect_tx(&full[slot], SM::kTile);
                         const CUtensorMap *map = kv ? &tm_v : &tm_k;
                         for (int hf = 0; hf < D / 64; ++hf)
-                            tma_load_4d(sRing + slot * SM::kTile + hf * SM::kHalf, map, &full[slot], hf * 64, kvh,
-                                        j * kPfKeys, b);
+                            tma_load_4d(dst + hf * SM::kHalf, map, &full[slot], hf * 64, kvh, (j - n_past) * kPfKeys, b);
                     }
                 }
-                if (*abort_flag) {   // let the copies in flight land before TMEM and smem go away
-                    mbar_wait_drain(qfull, 0, p.status);
-                    for (int i = max(0, item - kPfRing); i < item; ++i)
-                        mbar_wait_drain(&full[i % kPfRing], (i / kPfRing) & 1, p.status);
-                }
+            }
+            if (lane == 0 && *abort_flag) {   // let the copies in flight land before TMEM and smem go away
+                mbar_wait_drain(qfull, 0, p.status);
+                for (int i = max(0, item - kPfRing); i < item; ++i)
+                    mbar_wait_drain(&full[i % kPfRing], (i / kPfRing) & 1, p.status);
             }
             __syncwarp();
         } else if (warp == 9) {
@@ -204,6 +292,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         if (!v_ready) {
                             if (!ready(2 * j + 1)) { ok = false; continue; }
                             v_ready = true;
+                            if (PAGED && j == n_past - 1 && (past % kPfKeys) != 0) {
+                                // V rows past the cached tokens hold whatever the pages hold: zero them
+                                uint8_t *vt = sRing + ((2 * j + 1) % kPfRing) * SM::kTile;
+                                for (int hf = 0; hf < D / 64; ++hf)
+                                    for (int r = past % kPfKeys; r < kPfKeys; ++r) {
+                                        uint4 *row = reinterpret_cast<uint4 *>(vt + hf * SM::kHalf + r * 128);
+#pragma unroll
+                                        for (int c = 0; c < 8; ++c) row[c] = make_uint4(0u, 0u, 0u, 0u);
+                                    }
+                                fence_proxy_async_smem();   // generic-proxy stores before the tensor core reads
+                            }
                         }
                         issue_pv(t, 2 * j + 1, j > 0);
                         if (j + 1 < n_t) {
@@ -226,6 +325,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 }
             }
             __syncwarp();
+        } else if (PAGED && head % p.G == 0) {
+            // ------------------------------------------------------------ the append (warps 10, 11)
+            // rows of this CTA's two query tiles -> cache positions past + row, K and V
+            constexpr int CH = D * 2 / 16;   // 16-byte chunks per row
+            const int w = threadIdx.x - 10 * 32;
+            const int r0 = q0, r1 = min(q0 + 2 * kPfRows, p.S_q);
+            const size_t row_elems = static_cast<size_t>(p.n_kv) * D;
+            for (int it = w; it < (r1 - r0) * CH; it += 64) {
+                const int t = r0 + it / CH, c = it % CH;
+                const int pos = past + t;
+                const int page = p.block_table[static_cast<size_t>(b) * p.max_blocks + pos / p.page_size];
+                if (page < 0 || page >= p.num_pages) {
+                    record_status(p.status, kStatusInvalid);
+                    continue;
+                }
+                const size_t src = (static_cast<size_t>(b) * p.S_q + t) * row_elems + static_cast<size_t>(kvh) * D + c * 8;
+                const size_t dst = (static_cast<size_t>(page) * p.page_size + pos % p.page_size) * row_elems +
+                                   static_cast<size_t>(kvh) * D + c * 8;
+                *reinterpret_cast<uint4 *>(p.k_pages + dst) = *reinterpret_cast<const uint4 *>(p.k_new + src);
+                *reinterpret_cast<uint4 *>(p.v_pages + dst) = *reinterpret_cast<const uint4 *>(p.v_new + src);
+            }
         }
     } else {
         regs_inc<kRegsSoftmax>();
@@ -235,7 +355,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int n_t = t ? n_t1 : n_t0;
         const int r = quad * 32 + lane;             // row within the tile == TMEM lane
         const int row = q0 + t * kPfRows + r;       // absolute query row
-        const int limit = p.causal ? min(p.S_kv - 1, row + (p.S_kv - p.S_q)) : p.S_kv - 1;
+        const int limit = p.causal ? min(p.S_kv - 1, row + (p.S_kv - p.S_q)) : p.S_kv - 1;   // (not PAGED)
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const uint32_t tS = tmem + t * 128 + lane_off;
         const uint32_t tO = tmem + 256 + t * D + lane_off;
@@ -246,9 +366,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const bool landed = mbar_wait(&sfull[t], j & 1, abort_flag, p.status);
             if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }   // tcgen05.ld/st are warp-aligned
             tc_fence_after();
-            // the whole S row of this thread, read once
-            const int key0 = j * kPfKeys;
-            const bool masked = key0 + kPfKeys - 1 > limit;
+            // the whole S row of this thread, read once.  Columns c <= lim_c are visible:
+            // PAGED past tile: cached tokens below `past`; chunk tile: causal within the chunk
+            const int lim_c = !PAGED ? limit - j * kPfKeys
+                              : j < n_past ? past - 1 - j * kPfKeys
+                                           : row - (j - n_past) * kPfKeys;
+            const bool masked = lim_c < kPfKeys - 1;
             static_assert(kPfKeys == 128, "four 32-column TMEM loads per row");
             uint32_t r0[32], r1[32], r2[32], r3[32];
             tmem_ld32(tS, r0);
@@ -273,7 +396,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 mx = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < kPfKeys; ++c)
-                    if (key0 + c <= limit) mx = fmaxf(mx, __uint_as_float(GQA_S(c)));
+                    if (c <= lim_c) mx = fmaxf(mx, __uint_as_float(GQA_S(c)));
             }
             const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * cl2;
             if (j == 0) {
@@ -309,8 +432,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     const float2 x = ffma2_bcast(__uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)), cl2, -m_used);
                     uint32_t pp = pack_bf16x2(exp2f(x.x), exp2f(x.y));
                     if (masked) {   // masked keys add nothing (also when scale == 0)
-                        if (key0 + c > limit) pp &= 0xFFFF0000u;
-                        if (key0 + c + 1 > limit) pp &= 0x0000FFFFu;
+                        if (c > lim_c) pp &= 0xFFFF0000u;
+                        if (c + 1 > lim_c) pp &= 0x0000FFFFu;
                     }
                     pk[e] = pp;
                     rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(pp));
@@ -360,11 +483,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 // ---------------------------------------------------------------------------
 // host launcher
 
-template <int D>
-static int launch_prefill_t(const void *q, const void *k, const void *v, void *out, int B, int S_q, int S_kv, int h,
-                            int n_kv, int causal, float scale, cudaStream_t stream) {
+struct PrefillCall {
+    const void *q, *k, *v;          // PAGED: k, v = the chunk's new K/V [B, S_q, n_kv, D]
+    void *out;
+    int B, S_q, S_kv, h, n_kv, causal;
+    float scale;
+    cudaStream_t stream;
+    // PAGED only
+    void *k_pages, *v_pages;
+    const int32_t *block_table, *past_lens;
+    int max_blocks, page_size, num_pages;
+};
+
+template <int D, bool PAGED>
+static int launch_prefill_t(const PrefillCall &c) {
     using SM = PrefillSmem<D>;
-    auto kern = gqa_prefill_kernel<D>;
+    auto kern = gqa_prefill_kernel<D, PAGED>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 3;
     static unsigned long long attr_done = 0;   // one bit per device
@@ -373,46 +507,110 @@ static int launch_prefill_t(const void *q, const void *k, const void *v, void *o
             return 3;
         attr_done |= 1ull << dev;
     }
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tkp, tvp;
     const uint32_t box[4] = {64, 1, kPfRows, 1};
     {
-        const uint64_t dims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(h), static_cast<uint64_t>(S_q),
-                                  static_cast<uint64_t>(B)};
-        const uint64_t strides[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(h) * D * 2,
-                                     static_cast<uint64_t>(S_q) * h * D * 2};
-        if (!gqa_host::encode_tensor_map(&tq, q, 4, dims, strides, box)) return 3;
+        const uint64_t dims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(c.h), static_cast<uint64_t>(c.S_q),
+                                  static_cast<uint64_t>(c.B)};
+        const uint64_t strides[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(c.h) * D * 2,
+                                     static_cast<uint64_t>(c.S_q) * c.h * D * 2};
+        if (!gqa_host::encode_tensor_map(&tq, c.q, 4, dims, strides, box)) return 3;
     }
     {
-        const uint64_t dims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(n_kv), static_cast<uint64_t>(S_kv),
-                                  static_cast<uint64_t>(B)};
-        const uint64_t strides[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(n_kv) * D * 2,
-                                     static_cast<uint64_t>(S_kv) * n_kv * D * 2};
-        if (!gqa_host::encode_tensor_map(&tk, k, 4, dims, strides, box)) return 3;
-        if (!gqa_host::encode_tensor_map(&tv, v, 4, dims, strides, box)) return 3;
+        const int S = PAGED ? c.S_q : c.S_kv;
+        const uint64_t dims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(c.n_kv), static_cast<uint64_t>(S),
+                                  static_cast<uint64_t>(c.B)};
+        const uint64_t strides[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(c.n_kv) * D * 2,
+                                     static_cast<uint64_t>(S) * c.n_kv * D * 2};
+        if (!gqa_host::encode_tensor_map(&tk, c.k, 4, dims, strides, box)) return 3;
+        if (!gqa_host::encode_tensor_map(&tv, c.v, 4, dims, strides, box)) return 3;
     }
-    PrefillParams prm;
-    prm.out = static_cast<__nv_bfloat16 *>(out);
-    prm.B = B;
-    prm.S_q = S_q;
-    prm.S_kv = S_kv;
-    prm.h = h;
-    prm.n_kv = n_kv;
-    prm.G = h / n_kv;
-    prm.n_pairs = (S_q + 2 * kPfRows - 1) / (2 * kPfRows);
-    prm.causal = causal ? 1 : 0;
-    prm.scale_log2 = scale * 1.4426950408889634f;
+    if (PAGED) {
+        // [num_pages, page_size, n_kv, D]; page ids past num_pages read as zeros
+        const uint64_t dims[4] = {static_cast<uint64_t>(D), static_cast<uint64_t>(c.n_kv),
+                                  static_cast<uint64_t>(c.page_size), static_cast<uint64_t>(c.num_pages)};
+        const uint64_t strides[3] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(c.n_kv) * D * 2,
+                                     static_cast<uint64_t>(c.page_size) * c.n_kv * D * 2};
+        const uint32_t pbox[4] = {64, 1, static_cast<uint32_t>(std::min(c.page_size, kPfKeys)), 1};
+        if (!gqa_host::encode_tensor_map(&tkp, c.k_pages, 4, dims, strides, pbox)) return 3;
+        if (!gqa_host::encode_tensor_map(&tvp, c.v_pages, 4, dims, strides, pbox)) return 3;
+    } else {
+        tkp = tk;   // not read
+        tvp = tv;
+    }
+    PrefillParams prm = {};
+    prm.out = static_cast<__nv_bfloat16 *>(c.out);
+    prm.B = c.B;
+    prm.S_q = c.S_q;
+    prm.S_kv = c.S_kv;
+    prm.h = c.h;
+    prm.n_kv = c.n_kv;
+    prm.G = c.h / c.n_kv;
+    prm.n_pairs = (c.S_q + 2 * kPfRows - 1) / (2 * kPfRows);
+    prm.causal = c.causal ? 1 : 0;
+    prm.scale_log2 = c.scale * 1.4426950408889634f;
     prm.status = gqa_host::device_status();
     if (!prm.status) return 3;
-    const long ctas = static_cast<long>(prm.n_pairs) * B * h;
+    prm.block_table = c.block_table;
+    prm.past_lens = c.past_lens;
+    prm.k_new = static_cast<const __nv_bfloat16 *>(c.k);
+    prm.v_new = static_cast<const __nv_bfloat16 *>(c.v);
+    prm.k_pages = static_cast<__nv_bfloat16 *>(c.k_pages);
+    prm.v_pages = static_cast<__nv_bfloat16 *>(c.v_pages);
+    prm.max_blocks = c.max_blocks;
+    prm.page_size = c.page_size;
+    prm.num_pages = c.num_pages;
+    const long ctas = static_cast<long>(prm.n_pairs) * c.B * c.h;
     if (ctas > 0x7fffffffL) return 1;
-    gqa_prefill_kernel<D><<<static_cast<unsigned>(ctas), kPfThreads, SM::kTotal, stream>>>(tq, tk, tv, prm);
+    kern<<<static_cast<unsigned>(ctas), kPfThreads, SM::kTotal, c.stream>>>(tq, tk, tv, tkp, tvp, prm);
     return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }
 
 int launch_prefill(const void *q, const void *k, const void *v, void *out, int B, int S_q, int S_kv, int h, int n_kv,
                    int d, int causal, float scale, cudaStream_t stream) {
-    if (d == 128) return launch_prefill_t<128>(q, k, v, out, B, S_q, S_kv, h, n_kv, causal, scale, stream);
-    return launch_prefill_t<64>(q, k, v, out, B, S_q, S_kv, h, n_kv, causal, scale, stream);
+    PrefillCall c = {};
+    c.q = q;
+    c.k = k;
+    c.v = v;
+    c.out = out;
+    c.B = B;
+    c.S_q = S_q;
+    c.S_kv = S_kv;
+    c.h = h;
+    c.n_kv = n_kv;
+    c.causal = causal;
+    c.scale = scale;
+    c.stream = stream;
+    if (d == 128) return launch_prefill_t<128, false>(c);
+    return launch_prefill_t<64, false>(c);
+}
+
+int launch_prefill_paged(const void *q, const void *k_new, const void *v_new, void *k_pages, void *v_pages,
+                         const int32_t *block_table, int max_blocks, int page_size, int num_pages,
+                         const int32_t *past_lens, void *out, int B, int S_q, int h, int n_kv, int d, float scale,
+                         cudaStream_t stream) {
+    PrefillCall c = {};
+    c.q = q;
+    c.k = k_new;
+    c.v = v_new;
+    c.out = out;
+    c.B = B;
+    c.S_q = S_q;
+    c.S_kv = S_q;
+    c.h = h;
+    c.n_kv = n_kv;
+    c.causal = 1;
+    c.scale = scale;
+    c.stream = stream;
+    c.k_pages = k_pages;
+    c.v_pages = v_pages;
+    c.block_table = block_table;
+    c.past_lens = past_lens;
+    c.max_blocks = max_blocks;
+    c.page_size = page_size;
+    c.num_pages = num_pages;
+    if (d == 128) return launch_prefill_t<128, true>(c);
+    return launch_prefill_t<64, true>(c);
 }
 
 }  // namespace gqa

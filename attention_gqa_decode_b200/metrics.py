@@ -41,6 +41,13 @@ def prefill_flops(B: int, S_q: int, S_kv: int, h: int, d_h: int, causal: bool) -
     return 4 * B * h * d_h * visible_pairs(S_q, S_kv, causal)
 
 
+def chunk_prefill_flops(past_lens, S_q: int, h: int, d_h: int) -> int:
+    """Causal chunk after past_lens[b] cached tokens: row r sees past + r + 1 keys;
+    2 d_h flops for each of Q K^T and P V per (row, visible key, head)."""
+    pairs = sum(max(int(p), 0) * S_q + S_q * (S_q + 1) // 2 for p in past_lens)
+    return 4 * h * d_h * pairs
+
+
 def prefill_io_bytes(B: int, S_q: int, S_kv: int, h: int, n_kv: int, d_h: int, elem_bytes: int = 2) -> int:
     """Compulsory HBM bytes: read Q, K, V once, write O once."""
     return elem_bytes * d_h * B * (2 * S_q * h + 2 * S_kv * n_kv)

@@ -277,6 +277,37 @@ def cache_variant_leg(kind, args, device, world, page_size=64):
     return {"kv_bytes": kv_bytes, "kernel_ms": kern_ms, "steps": steps, "copies": copies}
 
 
+def chunk_prefill_leg(args, device, world):
+    """The last 512-token chunk of B=4 sequences of 4096 tokens (h=32, n_kv=8, d=128):
+    3584 past tokens in 64-token pages (seeded random order), append + causal
+    attention in one launch.  Each step restores nothing: the append rewrites the
+    same slots with the same values."""
+    import torch
+    import attention_gqa_decode_b200 as gqa
+    from attention_gqa_decode_b200 import inputs, metrics
+    B, S_q, P, h, n_kv, d, ps = 4, 512, 3584, 32, 8, 128, 64
+    q, kn, vn, kp, vp, bt, past = inputs.chunk_prefill_inputs(4, B, S_q, [P] * B, h, n_kv, d, ps)
+    flops = metrics.chunk_prefill_flops([P] * B, S_q, h, d)
+    qd, knd, vnd, kpd, vpd, btd, pd = (t.to(device) for t in (q, kn, vn, kp, vp, bt, past))
+    out = torch.empty_like(qd)
+    stream = torch.cuda.current_stream(device)
+    scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)   # > L2: flushed between steps
+
+    def flush(i):
+        scratch.fill_(i & 0xFF)
+
+    steps = max(3, min(args.steps, 30))
+    barrier(world)
+    per, _ = time_launches(lambda i: gqa.prefill_paged(qd, knd, vnd, kpd, vpd, btd, pd, out=out), steps,
+                           max(3, args.warmup), stream, flush=flush)
+    barrier(world)
+    kern_ms = multirank.max_over_ranks(statistics.mean(per), device)
+    if gqa.gqa_get_device_status() != 0:
+        raise RuntimeError("device status after the chunked prefill leg")
+    return {"flops": flops, "kernel_ms": kern_ms, "steps": steps,
+            "workload": f"chunked prefill B{B} S_q{S_q} past{P} h{h} n_kv{n_kv} d{d}, {ps}-token pages"}
+
+
 def prefill_leg(args, device, world):
     import torch
     import attention_gqa_decode_b200 as gqa
@@ -347,6 +378,7 @@ def main():
     clocks = ClockSampler(device)
     dec = decode_leg(args, device, world, clocks)
     pre = None if args.no_prefill else prefill_leg(args, device, world)
+    chunk = None if (args.no_prefill or args.no_variants) else chunk_prefill_leg(args, device, world)
     variants = {} if args.no_variants else {
         "decode_fp8": cache_variant_leg("fp8", args, device, world),
         "decode_paged": cache_variant_leg("paged", args, device, world),
@@ -377,6 +409,15 @@ def main():
                          "frac": tf / pk["bf16"], "frac_of_sustained": tf / pk["bf16_sustained"],
                          "traffic": kernel_traffic("gqa_prefill_kernel"),
                          "algorithmic_flops_per_launch": pre["flops"], "peak_source": pk["src"]}}
+    if chunk is not None:
+        tf = chunk["flops"] / (chunk["kernel_ms"] / 1e3) / 1e12
+        line["prefill_paged_chunk"] = {
+            "metric": "GQA causal prefill TFLOP/s", "workload": chunk["workload"], "value": world * tf,
+            "unit": "TFLOP/s", "ms_per_call": chunk["kernel_ms"], "steps": chunk["steps"],
+            "l2": "256 MiB buffer written between calls",
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16"], "unit": "TFLOP/s",
+                         "frac": tf / pk["bf16"], "traffic": kernel_traffic("gqa_prefill_kernel[paged]"),
+                         "algorithmic_flops_per_launch": chunk["flops"], "peak_source": pk["src"]}}
     desc = {"decode_fp8": ("E4M3 cache, one fp32 scale per KV head", "gqa_decode_kernel[e4m3]"),
             "decode_paged": ("bf16 cache in 64-token pages, seeded random page order", "gqa_decode_kernel[paged]"),
             "decode_paged_fp8": ("E4M3 cache in 64-token pages", "gqa_decode_kernel[paged,e4m3]")}

@@ -161,6 +161,40 @@ int gqa_decode_paged_fp8(const void *q, const void *k_pages, const void *v_pages
                          const int32_t *seqlens, void *out,
                          int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
 
+/*
+ * Chunked prefill over a paged bf16 cache, with the append
+ * ("Evolution of AI Attention Mechanisms" (toolsku), "MHA Implementation":
+ * the new K/V are concatenated after the past ones; "Multi-Query Attention
+ * (MQA)" (inferensys glossary), "PagedAttention").
+ *   q               [B, S_q, h, d_h]        bf16  the chunk's queries
+ *   k_new, v_new    [B, S_q, n_kv, d_h]     bf16  the chunk's keys and values
+ *   k_pages, v_pages [num_pages, page_size, n_kv, d_h]  bf16  the cache, as in
+ *                   gqa_decode_paged; WRITTEN: row t of k_new[b] / v_new[b]
+ *                   goes to position past_lens[b] + t of sequence b (every KV
+ *                   head).  Slots at other positions are not touched.
+ *   block_table     [B, max_blocks]  int32  DEVICE array; must cover positions
+ *                   0 .. past_lens[b] + S_q - 1 of every sequence
+ *   past_lens       [B]  int32  DEVICE array: tokens already cached per
+ *                   sequence (<= 0: none)
+ *   out             [B, S_q, h, d_h]        bf16
+ * Query row r of sequence b sits at position past_lens[b] + r and attends to
+ * the keys at positions <= past_lens[b] + r (bottom-right causal), the past
+ * ones read from the pages and the chunk's from k_new / v_new.  The caller
+ * must not read or write the pages of these sequences until the stream
+ * reaches the call.  A page id outside [0, num_pages) or past_lens[b] + S_q
+ * above max_blocks * page_size is recorded as GQA_ERR_INVALID_ARG in the
+ * device status word (such pages read as zeros and are not written; such a
+ * past length is cut).
+ * Errors: as gqa_prefill (pointers, sizes, scale, d_h) and gqa_decode_paged
+ * (block_table, max_blocks, page_size, num_pages), plus GQA_ERR_INVALID_ARG
+ * for S_q > max_blocks * page_size.
+ */
+int gqa_prefill_paged(const void *q, const void *k_new, const void *v_new,
+                      void *k_pages, void *v_pages,
+                      const int32_t *block_table, int max_blocks, int page_size, int num_pages,
+                      const int32_t *past_lens, void *out,
+                      int B, int S_q, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
+
 /* A static, human-readable name for a gqa_status_t value. */
 const char *gqa_status_string(int status);
 

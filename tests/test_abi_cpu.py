@@ -131,3 +131,18 @@ def test_binding_rejects_bad_cache_dtypes():
     k = torch.zeros(8, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(TypeError):       # bf16 codes for an 8-bit cache
         gqa.decode_fp8(q, k, k, None, None, None)
+
+
+@pytest.mark.parametrize("args,expect", [
+    # q, k_new, v_new, k_pages, v_pages, table, max_blocks, page_size, num_pages, past, out, B, S_q, h, n_kv, d, scale
+    ((0, A, A, A, A, A, 4, 64, 10, A, A, 2, 8, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),      # null q
+    ((A, A, A, A, A, A, 4, 64, 10, 0, A, 2, 8, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),      # null past_lens
+    ((A, A, A, BAD, A, A, 4, 64, 10, A, A, 2, 8, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),    # misaligned pages
+    ((A, A, A, A, A, A, 4, 48, 10, A, A, 2, 8, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),      # page size
+    ((A, A, A, A, A, A, 1, 64, 10, A, A, 2, 65, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),     # chunk > table
+    ((A, A, A, A, A, A, 4, 64, 10, A, A, 2, 8, 4, 3, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),      # h % n_kv
+    ((A, A, A, A, A, A, 4, 64, 10, A, A, 2, 8, 4, 2, 128, -1.0), _lib.GQA_ERR_INVALID_ARG),     # scale
+    ((A, A, A, A, A, A, 4, 64, 10, A, A, 2, 8, 4, 2, 80, 0.1), _lib.GQA_ERR_UNSUPPORTED),       # d_h
+])
+def test_prefill_paged_rejects(L, args, expect):
+    assert gqa.gqa_prefill_paged(*args, None) == expect

@@ -1,8 +1,8 @@
 """8-bit (E4M3) and paged decode caches: the CUDA path through the C ABI
 against the fp64 oracle.
 
-Tolerance as for the bf16 path: max |GPU - oracle| <= 1e-2 and mean
-|GPU - oracle| <= 1e-3 per call.  The oracle reads the same codes and scales,
+Tolerance as for the bf16 path (tests/_tol.py): max |GPU - oracle| <= 1e-2,
+or one bf16 step where |oracle| >= 2, and mean |GPU - oracle| <= 1e-3 per call.  The oracle reads the same codes and scales,
 so quantisation error is not part of the comparison: only the kernel's own
 rounding (Q to f16, weights to f16, fp32 sums, bf16 output) is.
 """
@@ -14,19 +14,9 @@ import attention_gqa_decode_b200 as gqa
 import oracle
 from attention_gqa_decode_b200 import _lib, inputs
 
+from tests._tol import MAX_ABS, MEAN_ABS, check  # noqa: F401
+
 pytestmark = pytest.mark.gpu
-
-MAX_ABS = 1e-2
-MEAN_ABS = 1e-3
-
-
-def check(got: torch.Tensor, ref: np.ndarray, what: str):
-    g = got.detach().float().cpu().double().numpy()
-    assert g.shape == ref.shape, (g.shape, ref.shape)
-    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
-    err = np.abs(g - ref)
-    mx, mean = float(err.max()), float(err.mean())
-    assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max abs {mx:.3e}, mean abs {mean:.3e}"
 
 
 def gpu_fp8(q, kc, vc, ks, vs, lens, scale=None):
