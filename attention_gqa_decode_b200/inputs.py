@@ -214,3 +214,23 @@ def chunk_prefill_inputs(seed: int, B: int, S_q: int, past_lens, h: int, n_kv: i
     v_new = _randn_bf16(g, (B, S_q, n_kv, d))
     kp, vp, bt = page_caches(seed + 1, k_past, v_past, past, page_size, spare_pages=spare_pages, reserve=S_q)
     return q, k_new, v_new, kp, vp, bt, past
+
+
+def mla_decode_inputs(seed: int, B: int, h: int, d_c: int, seqlens):
+    """q_absorbed [B,h,d_c] and the packed latent cache c_kv [sum(seqlens), d_c], bf16.
+
+    The absorbed query stands for q W_k_up of a trained model; with no weights here
+    it is drawn directly, N(0,1) like the other inputs (cache first, then queries).
+    """
+    if isinstance(seqlens, int):
+        seqlens = torch.full((B,), seqlens, dtype=torch.int32)
+    seqlens = torch.as_tensor(seqlens, dtype=torch.int32).reshape(B)
+    total = int(seqlens.clamp(min=0).sum())
+    g = _gen(seed)
+    c = _randn_bf16(g, (total, d_c))
+    q = _randn_bf16(g, (B, h, d_c))
+    return q, c, seqlens
+
+
+MLA_DECODE = Workload("MLA absorbed decode B16 h32 d_c512 L4096", "decode", 6, B=16, h=32, n_kv=1, d=512,
+                      kv_len=4096, notes="latent cache shared by all heads; K = V = c_kv")

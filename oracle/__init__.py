@@ -246,3 +246,22 @@ def prefill_paged(q, k_new, v_new, k_pages, v_pages, block_table, past_lens, sca
     if rc:
         raise ValueError("oracle_prefill_paged rejected its arguments")
     return out, kp, vp
+
+
+def mla_decode(q_absorbed, c_kv, seqlens, scale: float | None = None, n_threads: int = 0) -> np.ndarray:
+    """Absorbed multi-head latent attention decode; returns fp64 [B,h,d_c].
+
+    "Evolution of AI Attention Mechanisms" (toolsku), "Generation 3: MLA Multi-Head
+    Latent Attention": the cache holds one shared latent c_kv per token; with the key
+    up-projection absorbed into the query (q' = q W_k_up), the scores are
+    q' c_kv^T * scale and the weights multiply c_kv itself.  So this is the plain
+    decode of one KV head whose keys and values are both c_kv: q_absorbed
+    [B,h,d_c], c_kv packed [sum(seqlens), d_c].  ``scale=None`` is d_c ** -0.5, the
+    factor of that page's code.
+    """
+    cb = _bits(c_kv)
+    d_c = cb.shape[-1]
+    c3 = cb.reshape(-1, 1, d_c)
+    if scale is None:
+        scale = float(d_c) ** -0.5
+    return decode_general(q_absorbed, c3, c3, seqlens, scale=scale, n_threads=n_threads)
