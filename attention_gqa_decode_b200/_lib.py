@@ -22,6 +22,7 @@ SIGNATURES = {
     "gqa_decode_paged": ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_paged_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_prefill_paged": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp], _i),
+    "gqa_mla_decode": ([_vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp], _i),
     "gqa_status_string": ([_i], ctypes.c_char_p),
     "gqa_get_device_status": ([_vp], _i),
 }
@@ -95,6 +96,10 @@ def gqa_prefill_paged(q, k_new, v_new, k_pages, v_pages, block_table, max_blocks
                       out, B, S_q, h, n_kv, d_h, scale, stream) -> int:
     return lib().gqa_prefill_paged(q, k_new, v_new, k_pages, v_pages, block_table, max_blocks, page_size, num_pages,
                                    past_lens, out, B, S_q, h, n_kv, d_h, float(scale), stream)
+
+
+def gqa_mla_decode(q_absorbed, c_kv, seqlens, out, B, h, d_c, scale, stream) -> int:
+    return lib().gqa_mla_decode(q_absorbed, c_kv, seqlens, out, B, h, d_c, float(scale), stream)
 
 
 def gqa_get_device_status(stream=None) -> int:
@@ -325,4 +330,30 @@ def prefill_paged(q, k_new, v_new, k_pages, v_pages, block_table, past_lens, sca
                                past_lens.data_ptr(), out.data_ptr(), B, S_q, h, n_kv, d, scale, _stream_ptr(stream))
     if st != GQA_OK:
         raise GQAError(st, "gqa_prefill_paged")
+    return out
+
+
+def mla_decode(q_absorbed, c_kv, seqlens, scale: float | None = None, out=None, stream=None):
+    """Absorbed MLA decode: q_absorbed [B,h,d_c], packed latent cache c_kv [sum(seqlens),d_c] (bf16,
+    CUDA), seqlens int32 [B].  Returns softmax(q' c^T * scale) c as bf16 [B,h,d_c];
+    ``scale=None`` is d_c ** -0.5."""
+    import torch
+    _check(q_absorbed, "q_absorbed", 3), _check(c_kv, "c_kv", 2)
+    B, h, d_c = q_absorbed.shape
+    if c_kv.shape[1] != d_c:
+        raise ValueError(f"latent width mismatch q{tuple(q_absorbed.shape)} c_kv{tuple(c_kv.shape)}")
+    _check_seqlens(seqlens, B)
+    if scale is None:
+        scale = float(d_c) ** -0.5
+    if out is None:
+        out = torch.empty_like(q_absorbed)
+    else:
+        _check(out, "out", 3)
+        if out.shape != q_absorbed.shape:
+            raise ValueError("out must have q_absorbed's shape")
+    with torch.cuda.device(q_absorbed.device):
+        st = gqa_mla_decode(q_absorbed.data_ptr(), c_kv.data_ptr(), seqlens.data_ptr(), out.data_ptr(), B, h, d_c,
+                            scale, _stream_ptr(stream))
+    if st != GQA_OK:
+        raise GQAError(st, "gqa_mla_decode")
     return out

@@ -11,7 +11,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["api.cu", "decode.cu", "prefill.cu"]
+SOURCES = ["api.cu", "decode.cu", "prefill.cu", "mla.cu"]
 HEADERS = ["common.cuh"]
 LIB = os.path.join(PKG, "libgqa_b200.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -18,6 +18,8 @@ int launch_prefill_paged(const void *q, const void *k_new, const void *v_new, vo
                          const int32_t *block_table, int max_blocks, int page_size, int num_pages,
                          const int32_t *past_lens, void *out, int B, int S_q, int h, int n_kv, int d, float scale,
                          cudaStream_t stream);
+int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h, float scale,
+                      cudaStream_t stream);
 int launch_decode_ex(const void *q, const void *k, const void *v, const float *k_scale, const float *v_scale,
                      const int32_t *seqlens, const int32_t *block_table, int max_blocks, int page_size,
                      int num_pages, void *out, int B, int h, int n_kv, int d, float scale, cudaStream_t stream);
@@ -201,6 +203,17 @@ int gqa_prefill_paged(const void *q, const void *k_new, const void *v_new, void 
     if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
     return gqa::launch_prefill_paged(q, k_new, v_new, k_pages, v_pages, block_table, max_blocks, page_size,
                                      num_pages, past_lens, out, B, S_q, h, n_kv, d_h, scale, stream);
+}
+
+int gqa_mla_decode(const void *q_absorbed, const void *c_kv, const int32_t *seqlens, void *out, int B, int h,
+                   int d_c, float scale, cudaStream_t stream) {
+    if (!q_absorbed || !c_kv || !seqlens || !out) return GQA_ERR_INVALID_ARG;
+    if (!aligned16(q_absorbed) || !aligned16(c_kv) || !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+        return GQA_ERR_INVALID_ARG;
+    if (B <= 0 || B > 65535 || h <= 0 || h > 65535 * 16) return GQA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return GQA_ERR_INVALID_ARG;
+    if (d_c != 512) return GQA_ERR_UNSUPPORTED;
+    return gqa::launch_mla_decode(q_absorbed, c_kv, seqlens, out, B, h, scale, stream);
 }
 
 const char *gqa_status_string(int status) {

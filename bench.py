@@ -308,6 +308,31 @@ def chunk_prefill_leg(args, device, world):
             "workload": f"chunked prefill B{B} S_q{S_q} past{P} h{h} n_kv{n_kv} d{d}, {ps}-token pages"}
 
 
+def mla_leg(args, device, world):
+    """Absorbed MLA decode, B16 h32 d_c512 L4096 (64 MiB latent cache per step);
+    copies rotated so each step reads a cache L2 has not seen for several steps."""
+    import torch
+    import attention_gqa_decode_b200 as gqa
+    from attention_gqa_decode_b200 import inputs
+    w = inputs.MLA_DECODE
+    q, c, lens = inputs.mla_decode_inputs(w.seed, w.B, w.h, w.d, w.kv_len)
+    nbytes = c.numel() * c.element_size()
+    copies = max(3, -(-3 * 128 * 1024 * 1024 // nbytes))
+    qd, ld = q.to(device), lens.to(device)
+    cs = [c.to(device) for _ in range(copies)]
+    out = torch.empty_like(qd)
+    stream = torch.cuda.current_stream(device)
+    steps = max(3, min(args.steps, 300))
+    barrier(world)
+    per, _ = time_launches(lambda i: gqa.mla_decode(qd, cs[i % copies], ld, out=out), steps, max(3, args.warmup),
+                           stream)
+    barrier(world)
+    kern_ms = multirank.max_over_ranks(statistics.mean(per), device)
+    if gqa.gqa_get_device_status() != 0:
+        raise RuntimeError("device status after the MLA decode leg")
+    return {"kv_bytes": nbytes, "kernel_ms": kern_ms, "steps": steps, "copies": copies, "workload": w.name}
+
+
 def prefill_leg(args, device, world):
     import torch
     import attention_gqa_decode_b200 as gqa
@@ -379,6 +404,7 @@ def main():
     dec = decode_leg(args, device, world, clocks)
     pre = None if args.no_prefill else prefill_leg(args, device, world)
     chunk = None if (args.no_prefill or args.no_variants) else chunk_prefill_leg(args, device, world)
+    mla = None if args.no_variants else mla_leg(args, device, world)
     variants = {} if args.no_variants else {
         "decode_fp8": cache_variant_leg("fp8", args, device, world),
         "decode_paged": cache_variant_leg("paged", args, device, world),
@@ -418,6 +444,15 @@ def main():
             "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16"], "unit": "TFLOP/s",
                          "frac": tf / pk["bf16"], "traffic": kernel_traffic("gqa_prefill_kernel[paged]"),
                          "algorithmic_flops_per_launch": chunk["flops"], "peak_source": pk["src"]}}
+    if mla is not None:
+        gbs = mla["kv_bytes"] / (mla["kernel_ms"] / 1e3) / 1e9
+        line["mla_decode"] = {
+            "metric": "MLA decode latent-cache GB/s", "workload": mla["workload"], "value": world * gbs,
+            "unit": "GB/s", "ms_per_call": mla["kernel_ms"], "steps": mla["steps"],
+            "tokens_per_s": world * 16 / (mla["kernel_ms"] / 1e3), "l2": f"{mla['copies']} cache copies rotated",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
+                         "traffic": kernel_traffic("gqa_mla_decode_kernel"),
+                         "algorithmic_bytes_per_launch": mla["kv_bytes"], "peak_source": pk["src"]}}
     desc = {"decode_fp8": ("E4M3 cache, one fp32 scale per KV head", "gqa_decode_kernel[e4m3]"),
             "decode_paged": ("bf16 cache in 64-token pages, seeded random page order", "gqa_decode_kernel[paged]"),
             "decode_paged_fp8": ("E4M3 cache in 64-token pages", "gqa_decode_kernel[paged,e4m3]")}

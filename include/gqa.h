@@ -195,6 +195,26 @@ int gqa_prefill_paged(const void *q, const void *k_new, const void *v_new,
                       const int32_t *past_lens, void *out,
                       int B, int S_q, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
 
+/*
+ * Absorbed multi-head latent attention (MLA) decode ("Evolution of AI
+ * Attention Mechanisms" (toolsku), "Generation 3: MLA Multi-Head Latent
+ * Attention": one latent vector c_kv per token is cached for all heads; with
+ * the key up-projection absorbed into the query, Q K^T = (Q W_k_up) c_kv^T,
+ * and the softmax weights multiply c_kv itself).
+ *   q_absorbed  [B, h, d_c]            bf16  q' = q W_k_up per head (the
+ *                                            caller's projection)
+ *   c_kv        [sum_b seqlens[b], d_c] bf16  packed latent cache, sequence b
+ *                                            starting at row sum_{b'<b} seqlens[b']
+ *   seqlens     [B]  int32  DEVICE array (<= 0: zero row)
+ *   out         [B, h, d_c]            bf16  softmax(q' c_kv^T * scale) c_kv
+ * d_c must be 512 (the pages' latent width); the pages' code uses
+ * scale = d_c^-0.5.  Errors: GQA_ERR_INVALID_ARG for null or misaligned
+ * pointers, B <= 0 or > 65535, h <= 0, a bad scale; GQA_ERR_UNSUPPORTED for
+ * d_c != 512.
+ */
+int gqa_mla_decode(const void *q_absorbed, const void *c_kv, const int32_t *seqlens, void *out,
+                   int B, int h, int d_c, float scale, cudaStream_t stream);
+
 /* A static, human-readable name for a gqa_status_t value. */
 const char *gqa_status_string(int status);
 

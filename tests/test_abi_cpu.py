@@ -146,3 +146,17 @@ def test_binding_rejects_bad_cache_dtypes():
 ])
 def test_prefill_paged_rejects(L, args, expect):
     assert gqa.gqa_prefill_paged(*args, None) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    # q_absorbed, c_kv, seqlens, out, B, h, d_c, scale
+    ((0, A, A, A, 2, 32, 512, 0.04), _lib.GQA_ERR_INVALID_ARG),
+    ((A, BAD, A, A, 2, 32, 512, 0.04), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A + 1, A, 2, 32, 512, 0.04), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, 0, 32, 512, 0.04), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, 2, 0, 512, 0.04), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, 2, 32, 512, float("nan")), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, A, 2, 32, 256, 0.04), _lib.GQA_ERR_UNSUPPORTED),
+])
+def test_mla_decode_rejects(L, args, expect):
+    assert gqa.gqa_mla_decode(*args, None) == expect
