@@ -7,9 +7,13 @@
     python -m attention_gqa_decode_b200.profile_case decode_paged64 GQA_DECODE_70B 3
     python -m attention_gqa_decode_b200.profile_case decode_paged64_fp8 GQA_DECODE_70B 3
 
+    python -m attention_gqa_decode_b200.profile_case mla MLA_DECODE 3
+    python -m attention_gqa_decode_b200.profile_case prefill_chunk GQA_CAUSAL_PREFILL 2
+
 ``decode_fp8`` stores the decode workload's caches as E4M3 codes (one scale
 per KV head); ``decode_paged<N>`` cuts them into pages of N tokens, and a
-``_fp8`` suffix does both.
+``_fp8`` suffix does both.  ``prefill_chunk`` runs the last 512-token chunk of
+the prefill workload's sequences (3584 past tokens in 64-token pages).
 
 The inputs are the seeded synthetic ones; nothing is checked or timed here.
 """
@@ -32,6 +36,24 @@ def main(argv) -> int:
     else:
         w = getattr(inputs, name)
     base = kind.split("_")[0]
+    if kind == "mla":
+        q, c, lens = (x.cuda() for x in inputs.mla_decode_inputs(w.seed, w.B, w.h, w.d, w.kv_len))
+        for _ in range(n):
+            gqa.mla_decode(q, c, lens)
+        torch.cuda.synchronize()
+        st = gqa.gqa_get_device_status()
+        print(f"{w.name}: {n} calls, device status {st}")
+        return 0 if st == 0 else 1
+    if kind == "prefill_chunk":
+        S_q, P = 512, w.S_q - 512
+        t = inputs.chunk_prefill_inputs(w.seed, w.B, S_q, [P] * w.B, w.h, w.n_kv, w.d, 64)
+        q, kn, vn, kp, vp, bt, past = (x.cuda() for x in t)
+        for _ in range(n):
+            gqa.prefill_paged(q, kn, vn, kp, vp, bt, past)
+        torch.cuda.synchronize()
+        st = gqa.gqa_get_device_status()
+        print(f"{w.name} last chunk: {n} calls, device status {st}")
+        return 0 if st == 0 else 1
     if base != w.kind:
         raise SystemExit(f"{name} is a {w.kind} workload")
     fp8 = kind.endswith("_fp8")
