@@ -433,11 +433,13 @@ __global__ void __launch_bounds__(kDecThreads, MINB)
     if (warp == kDecWarps) {
         // ------------------------------------------------------------ producer
         const int pb = PAGED ? min(p.page_size, TOK) : TOK;   // tokens per TMA box
-        // paged: lane j < boxes(i) holds the page id of box j of stage i
-        auto page_of = [&](int i) -> int {
-            const int t = (first + i) * TOK + lane * pb;
+        const int pieces = TOK / pb;                           // boxes per stage
+        // paged: box k of stage i is piece n = i * pieces + k of this split; lane l
+        // holds the page id of piece 32 * batch + l, the next batch loaded a batch ahead
+        auto batch_of = [&](int batch) -> int {
+            const int t = first * TOK + (batch * 32 + lane) * pb;
             int page = 0;
-            if (lane * pb < TOK && t < L) {
+            if (PAGED && t < L) {
                 page = p.block_table[static_cast<size_t>(b) * p.max_blocks + t / p.page_size];
                 if (page < 0 || page >= p.num_pages) {   // read as zeros, reported
                     record_status(p.status, kStatusInvalid);
@@ -446,7 +448,9 @@ __global__ void __launch_bounds__(kDecThreads, MINB)
             }
             return page;
         };
-        int next_pages = (PAGED && n_stages > 0) ? page_of(0) : 0;
+        int cur_batch = 0;
+        int ids = (PAGED && n_stages > 0) ? batch_of(0) : 0;
+        int ids_next = (PAGED && n_stages * pieces > 32) ? batch_of(1) : 0;
         int issued = 0;
         for (int i = 0; i < n_stages; ++i) {
             const int slot = i % STAGES, use = i / STAGES;
@@ -469,13 +473,17 @@ __global__ void __launch_bounds__(kDecThreads, MINB)
                     }
                 }
             } else {
-                const int pages = next_pages;
-                if (i + 1 < n_stages) next_pages = page_of(i + 1);
                 const int nb = (min(TOK, L - t0) + pb - 1) / pb;   // boxes of this stage
                 if (lane == 0)
                     mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nb * pb * RB * Geo::kPanels * 2));
                 for (int j = 0; j < nb; ++j) {
-                    const int page = __shfl_sync(0xffffffffu, pages, j);
+                    const int n = i * pieces + j;
+                    if (n / 32 != cur_batch) {   // warp-uniform
+                        cur_batch = n / 32;
+                        ids = ids_next;
+                        if ((cur_batch + 1) * 32 < n_stages * pieces) ids_next = batch_of(cur_batch + 1);
+                    }
+                    const int page = __shfl_sync(0xffffffffu, ids, n % 32);
                     if (lane == 0) {
                         const int slot_in_page = (t0 + j * pb) % p.page_size;
 #pragma unroll

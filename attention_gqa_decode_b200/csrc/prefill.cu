@@ -186,11 +186,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         tma_load_4d(sQ + t * SM::kTile + hf * SM::kHalf, &tm_q, qfull, hf * 64, head, q0 + t * kPfRows, b);
             }
             const int pb = PAGED ? min(p.page_size, kPfKeys) : kPfKeys;   // rows per page box
-            // lane k: page id of piece k of past tile j (0 where there is none)
-            auto page_of = [&](int j) -> int {
+            const int pieces = kPfKeys / pb;                               // boxes per past tile
+            // piece n = j * pieces + k covers past rows [n pb, n pb + pb); lane l holds the
+            // page id of piece 32 * batch + l, the next batch loaded a batch ahead
+            auto batch_of = [&](int batch) -> int {
                 int page = 0;
-                const int pos = j * kPfKeys + lane * pb;
-                if (PAGED && j < n_past && lane * pb < kPfKeys && pos < past) {
+                const int pos = (batch * 32 + lane) * pb;
+                if (PAGED && pos < past) {
                     page = p.block_table[static_cast<size_t>(b) * p.max_blocks + pos / p.page_size];
                     if (page < 0 || page >= p.num_pages) {   // read as zeros, reported
                         record_status(p.status, kStatusInvalid);
@@ -199,12 +201,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 }
                 return page;
             };
-            int next_pages = page_of(0);
+            int cur_batch = 0;
+            int ids = PAGED ? batch_of(0) : 0;
+            int ids_next = (PAGED && n_past * pieces > 32) ? batch_of(1) : 0;
             int item = 0;
             bool stop = false;
             for (int j = 0; j < nmax && !stop; ++j) {
-                const int pages = next_pages;
-                if (PAGED && j + 1 < nmax) next_pages = page_of(j + 1);
                 for (int kv = 0; kv < 2; ++kv, ++item) {
                     const int slot = item % kPfRing, use = item / kPfRing;
                     int ok = 1;
@@ -221,7 +223,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         const CUtensorMap *map = kv ? &tm_vp : &tm_kp;
                         if (lane == 0) mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nb * pb * 128 * (D / 64)));
                         for (int k = 0; k < nb; ++k) {
-                            const int page = __shfl_sync(0xffffffffu, pages, k);
+                            const int n = j * pieces + k;
+                            if (n / 32 != cur_batch) {   // warp-uniform
+                                cur_batch = n / 32;
+                                ids = ids_next;
+                                if ((cur_batch + 1) * 32 < n_past * pieces) ids_next = batch_of(cur_batch + 1);
+                            }
+                            const int page = __shfl_sync(0xffffffffu, ids, n % 32);
                             if (lane == 0) {
                                 const int slot_in_page = (j * kPfKeys + k * pb) % p.page_size;
                                 for (int hf = 0; hf < D / 64; ++hf)
