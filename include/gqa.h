@@ -47,7 +47,7 @@ extern "C" {
 typedef enum {
     GQA_OK = 0,
     GQA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, h % n_kv != 0, bad scale */
-    GQA_ERR_UNSUPPORTED = 2,   /* a valid request this build does not implement (d_h not 64/128) */
+    GQA_ERR_UNSUPPORTED = 2,   /* a valid request the library does not implement (e.g. d_h not 64/128) */
     GQA_ERR_CUDA = 3,          /* the launch failed (see cudaGetLastError) */
     GQA_ERR_TIMEOUT = 4        /* a kernel gave up on an internal wait (device status only) */
 } gqa_status_t;
