@@ -18,11 +18,14 @@ def run(q, c, lens, scale=None):
 
 
 @pytest.mark.parametrize("B,h,lens", [
-    (3, 32, [1, 31, 33]),            # around the 32-token stage
+    (3, 32, [1, 31, 33]),
+    (4, 32, [63, 64, 65, 129]),      # around 64 and 128 tokens
+    (3, 8, [127, 128, 4097]),        # a partial head group; a ragged long sequence
     (2, 16, [1000, 5000]),
-    (2, 128, [300, 2000]),           # eight 16-head groups
+    (2, 128, [300, 2000]),           # several head groups
     (3, 40, [64, 0, 7]),             # a partial head group, an empty sequence
     (1, 32, [20000]),                # long: eight splits
+    (1, 96, [9000]),                 # several head groups, several splits each
 ], ids=str)
 def test_mla_parity(B, h, lens):
     q, c, lens = inputs.mla_decode_inputs(60 + h, B, h, 512, lens)
@@ -51,3 +54,33 @@ def test_mla_single_token_is_exact():
 def test_mla_default_scale():
     q, c, lens = inputs.mla_decode_inputs(9, 2, 16, 512, [100, 50])
     assert torch.equal(run(q, c, lens), run(q, c, lens, scale=512 ** -0.5))
+
+
+def test_mla_nan_in_previous_sequence_stays_there():
+    # sequence 1 (30 tokens) is shorter than a stage: the box the kernel reads for it
+    # ends at its last token and starts inside sequence 0, whose last row holds a NaN
+    q, c, lens = inputs.mla_decode_inputs(10, 2, 32, 512, [100, 30])
+    c = c.clone()
+    c[99, 5] = float("nan")
+    got = run(q, c, lens)
+    assert torch.isnan(got[0].float()).any()
+    check(got[1:], oracle.mla_decode(q[1:], c[100:], lens[1:]), "sequence after a NaN row")
+
+
+def spiked_inputs(seed, B, h, lens):
+    """Latent rows along head 0's query, growing every 64 tokens for five stages, so
+    that head 0's running max jumps by more than 2^8 several times (the lazy rescale)."""
+    q, c, L = inputs.mla_decode_inputs(seed, B, h, 512, lens)
+    c = c.float()
+    off = 0
+    for b in range(B):
+        u = q[b, 0].float() / q[b, 0].float().norm()
+        for k in range(1, min(6, (int(L[b]) - 8) // 64 + 1)):
+            c[off + 64 * k + 7] = u * (6.0 * k)
+        off += int(L[b])
+    return q, c.to(torch.bfloat16), L
+
+
+def test_mla_running_max_rescale():
+    q, c, lens = spiked_inputs(70, 3, 32, [1000, 300, 2049])
+    check(run(q, c, lens), oracle.mla_decode(q, c, lens), "MLA with rescales")
