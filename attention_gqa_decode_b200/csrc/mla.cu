@@ -43,6 +43,7 @@ constexpr int kMlaPanels = kMlaDc / 64;           // 64-dim panels of 128-byte r
 constexpr int kMlaPanelBytes = kMlaTok * 128;
 constexpr int kMlaStageBytes = kMlaPanels * kMlaPanelBytes;   // 32 KB
 constexpr int kMlaMaxSplit = 8;
+constexpr float kMlaRescale = 8.0f;               // lazy rescale threshold (log2 units)
 
 struct MlaParams {
     const __nv_bfloat16 *q;
@@ -164,16 +165,8 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
         const uint32_t vrow = ((lane >> 3) & 1) * 8 + (lane & 7);   // P V: token within a 16-token k-step
         const uint32_t vchk = lane >> 4;                            //   which 8-dim n-tile of a pair
 
-        for (int i = 0; i < n_stages; ++i) {
-            const int slot = i % kMlaStages, use = i / kMlaStages;
-            const bool landed = mbar_wait(&full[slot], use & 1, abort_flag, p.status);
-            if (!__all_sync(0xffffffffu, landed)) break;
-            const int t0 = (first + i) * kMlaTok;
-            const int row_lo = max(0, t0 - (L - kMlaTok));   // rows of the box before this stage's tokens
-            const uint32_t stage = smem_u32(smem + slot * kMlaStageBytes);
-
-            // partial scores over this warp's 128 dims (16 heads x 32 tokens)
-            float s[NTS][4];
+        // partial scores over this warp's 128 dims (16 heads x 32 tokens) of the stage at `stage`
+        auto partial_scores = [&](uint32_t stage, float (&s)[NTS][4]) {
 #pragma unroll
             for (int nt = 0; nt < NTS; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
 #pragma unroll
@@ -189,17 +182,37 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
                     mma_bf16_16816(s[2 * np + 1], qa[ks], b2, b3);
                 }
             }
-            // sum the four partials: write ours once the previous stage's have been read
-            bool ok = true;
-            if (i > 0) ok = mbar_wait(sfree, (i - 1) & 1, abort_flag, p.status);
-            if (!__all_sync(0xffffffffu, ok)) break;
+        };
+        auto stage_addr = [&](int i) { return smem_u32(smem + (i % kMlaStages) * kMlaStageBytes); };
+        auto landed = [&](int i) {
+            return __all_sync(0xffffffffu, mbar_wait(&full[i % kMlaStages], (i / kMlaStages) & 1, abort_flag, p.status));
+        };
+
+        // Software-pipelined: the partial scores of stage i + 1 are computed between
+        // publishing this warp's partial of stage i and waiting for the other warps'.
+        float s[NTS][4];
+        bool ok = n_stages == 0 || landed(0);
+        if (ok && n_stages > 0) partial_scores(stage_addr(0), s);
+        for (int i = 0; i < n_stages && ok; ++i) {
+            const int slot = i % kMlaStages;
+            const int t0 = (first + i) * kMlaTok;
+            const int row_lo = max(0, t0 - (L - kMlaTok));   // rows of the box before this stage's tokens
+            const uint32_t stage = stage_addr(i);
+
+            // publish this warp's partial once every warp has read the previous stage's
+            if (i > 0 && !__all_sync(0xffffffffu, mbar_wait(sfree, (i - 1) & 1, abort_flag, p.status))) break;
 #pragma unroll
             for (int nt = 0; nt < NTS; ++nt)
                 sred[(warp * NTS + nt) * 32 + lane] = make_float4(s[nt][0], s[nt][1], s[nt][2], s[nt][3]);
             __syncwarp();
             if (lane == 0) mbar_arrive(sfull);
-            ok = mbar_wait(sfull, i & 1, abort_flag, p.status);
-            if (!__all_sync(0xffffffffu, ok)) break;
+            float sn[NTS][4];
+            if (i + 1 < n_stages) {
+                if (!landed(i + 1)) break;
+                partial_scores(stage_addr(i + 1), sn);
+            }
+            // the sum of the four partials (the same order in every warp)
+            if (!__all_sync(0xffffffffu, mbar_wait(sfull, i & 1, abort_flag, p.status))) break;
 #pragma unroll
             for (int nt = 0; nt < NTS; ++nt) {
                 float4 t = sred[nt * 32 + lane];
@@ -234,22 +247,36 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
                 mx[0] = fmax3(mx[0], s[nt][0], s[nt][1]);
                 mx[1] = fmax3(mx[1], s[nt][2], s[nt][3]);
             }
-            float alpha[2];
+            // lazy rescale: the running max moves only when a row's stage max exceeds it
+            // by 2^8 (every warp sees the same sums, so all take the same decisions)
+            float m_tile[2];
+            bool need = false;
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
                 mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-                const float m_new = fmaxf(m_run[r], mx[r] * cl2);   // >= 1 valid token per stage
-                alpha[r] = exp2f(m_run[r] - m_new);
-                m_run[r] = m_new;
-                l_run[r] *= alpha[r];
+                m_tile[r] = mx[r] * cl2;                             // >= 1 valid token per stage
+                need |= m_tile[r] > m_run[r] + kMlaRescale;
             }
+            if (i == 0) {
+                m_run[0] = m_tile[0];
+                m_run[1] = m_tile[1];
+            } else if (__any_sync(0xffffffffu, need)) {
+                float alpha[2];
 #pragma unroll
-            for (int nt = 0; nt < NT_O; ++nt) {
-                o[nt][0] *= alpha[0];
-                o[nt][1] *= alpha[0];
-                o[nt][2] *= alpha[1];
-                o[nt][3] *= alpha[1];
+                for (int r = 0; r < 2; ++r) {
+                    const float m_new = fmaxf(m_run[r], m_tile[r]);
+                    alpha[r] = exp2f(m_run[r] - m_new);
+                    m_run[r] = m_new;
+                    l_run[r] *= alpha[r];
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT_O; ++nt) {
+                    o[nt][0] *= alpha[0];
+                    o[nt][1] *= alpha[0];
+                    o[nt][2] *= alpha[1];
+                    o[nt][3] *= alpha[1];
+                }
             }
             uint32_t pa[KKS][4];
             float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
@@ -293,6 +320,13 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
+#pragma unroll
+            for (int nt = 0; nt < NTS; ++nt) {
+                s[nt][0] = sn[nt][0];
+                s[nt][1] = sn[nt][1];
+                s[nt][2] = sn[nt][2];
+                s[nt][3] = sn[nt][3];
+            }
         }
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
