@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace gqa {
 
 // ---------------------------------------------------------------------------
@@ -413,6 +415,20 @@ bool encode_tensor_map_ex(CUtensorMap *map, CUtensorMapDataType dtype, CUtensorM
                           const uint32_t *box);
 
 int sm_count();
+
+// Runs `set` (returning true on success) once per device for devices 0..63,
+// thread-safe; later calls on that device skip it.  Devices past 63 run it
+// every time.  Concurrent first calls may both run it, so it must be
+// idempotent (cudaFuncSetAttribute is).
+template <class F>
+bool once_per_device(std::atomic<unsigned long long> &done, int dev, F &&set) {
+    if (dev < 0 || dev >= 64) return set();
+    const unsigned long long bit = 1ull << dev;
+    if (done.load(std::memory_order_acquire) & bit) return true;
+    if (!set()) return false;
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    return true;
+}
 
 // Device address of the library's status word on the current device (null on failure).
 int *device_status();

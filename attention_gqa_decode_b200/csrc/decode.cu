@@ -882,15 +882,13 @@ static int launch_decode_t(const DecodeCall &c) {
     auto kern = gqa_decode_kernel<D, STAGES, WT, F, PAGED, TR, MINB>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 3;
-    static unsigned long long attr_done = 0;   // one bit per device
-    if (dev < 64 && !(attr_done >> dev & 1ull)) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal) != cudaSuccess)
-            return 3;
-        if (GQA_DECODE_MAX_SPLIT > 8 &&
-            cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-            return 3;
-        attr_done |= 1ull << dev;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    if (!gqa_host::once_per_device(attr_done, dev, [&] {
+            return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal) == cudaSuccess &&
+                   (GQA_DECODE_MAX_SPLIT <= 8 ||
+                    cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess);
+        }))
+        return 3;
     constexpr uint64_t E = Geo::kFp8 ? 1 : 2;   // bytes per element
     const CUtensorMapDataType dt = Geo::kFp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const CUtensorMapSwizzle swz = Geo::kRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;

@@ -401,12 +401,12 @@ int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, v
     auto kern = gqa_mla_decode_kernel;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 3;
-    static unsigned long long attr_done = 0;
-    if (dev < 64 && !(attr_done >> dev & 1ull)) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MlaSmem::kTotal) != cudaSuccess)
-            return 3;
-        attr_done |= 1ull << dev;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    if (!gqa_host::once_per_device(attr_done, dev, [&] {
+            return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MlaSmem::kTotal) ==
+                   cudaSuccess;
+        }))
+        return 3;
     CUtensorMap tc;
     const uint64_t dims[2] = {static_cast<uint64_t>(kMlaDc), 1ull << 30};   // token extent left open
     const uint64_t strides[1] = {static_cast<uint64_t>(kMlaDc) * 2};

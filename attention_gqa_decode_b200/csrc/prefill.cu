@@ -509,12 +509,11 @@ static int launch_prefill_t(const PrefillCall &c) {
     auto kern = gqa_prefill_kernel<D, PAGED>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 3;
-    static unsigned long long attr_done = 0;   // one bit per device
-    if (dev < 64 && !(attr_done >> dev & 1ull)) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal) != cudaSuccess)
-            return 3;
-        attr_done |= 1ull << dev;
-    }
+    static std::atomic<unsigned long long> attr_done{0};
+    if (!gqa_host::once_per_device(attr_done, dev, [&] {
+            return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal) == cudaSuccess;
+        }))
+        return 3;
     CUtensorMap tq, tk, tv, tkp, tvp;
     const uint32_t box[4] = {64, 1, kPfRows, 1};
     {
