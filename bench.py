@@ -127,8 +127,13 @@ def barrier(world):
 # ----------------------------------------------------------------------------
 # CPU legs (the oracle, as it stands, on the host cores)
 
-def oracle_decode_leg(target_s: float = 10.0):
-    """Time the fp64 oracle on whole sequences of the decode workload until ~target_s."""
+def oracle_decode_leg(target_s: float = 10.0, gpu_out=None):
+    """Time the fp64 oracle on whole sequences of the decode workload until ~target_s.
+
+    With `gpu_out` (the decode leg's bf16 result for the same seeded inputs) every
+    output of the sequences the oracle computed is also compared with it; the
+    comparison is returned as a second dict (None without `gpu_out`)."""
+    import numpy as np
     import oracle
     import torch
     from attention_gqa_decode_b200 import inputs, metrics
@@ -138,6 +143,7 @@ def oracle_decode_leg(target_s: float = 10.0):
     cores = os.cpu_count() or 1
     done_bytes, t_total, seqs = 0, 0.0, 0
     b = 0
+    errs, ulps, over, seen = [], [], 0, set()
     while t_total < target_s and seqs < 4 * w.B:
         nb = min(cores, w.B)                      # one batch of sequences per call, all cores
         b0 = (b * nb) % w.B
@@ -147,14 +153,35 @@ def oracle_decode_leg(target_s: float = 10.0):
         vs = torch.cat([v[j * per_seq:(j + 1) * per_seq] for j in idx]).contiguous()
         ls = lens[idx].contiguous()
         t0 = time.perf_counter()
-        oracle.decode(qs, ks, vs, ls, n_threads=cores)
+        ref = oracle.decode(qs, ks, vs, ls, n_threads=cores)
         t_total += time.perf_counter() - t0
         done_bytes += metrics.decode_kv_bytes(ls.tolist(), w.n_kv, w.d)
         seqs += nb
         b += 1
-    return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{seqs} whole sequences of the decode workload ({w.kv_len} tokens, h={w.h}, n_kv={w.n_kv}), "
-                      f"{t_total:.1f} s of fp64 oracle time"}
+        fresh = [i for i, j in enumerate(idx) if j not in seen]   # each sequence compared once
+        if gpu_out is not None and fresh:
+            seen.update(idx[i] for i in fresh)
+            got = gpu_out[[idx[i] for i in fresh]].double().numpy()
+            ref = ref[fresh]
+            err = np.abs(got - ref)
+            # one bf16 step around |ref| (normal range): 2^(floor(log2 |ref|) - 7)
+            step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 7)
+            bound = np.maximum(1e-2, step)
+            errs.append(err.ravel())
+            ulps.append((err / bound).ravel())
+            over += int((err > bound).sum())
+    cpu = {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+           "sample": f"{seqs} whole sequences of the decode workload ({w.kv_len} tokens, h={w.h}, n_kv={w.n_kv}), "
+                     f"{t_total:.1f} s of fp64 oracle time"}
+    if not errs:
+        return cpu, None
+    e, u = np.concatenate(errs), np.concatenate(ulps)
+    parity = {"outputs": int(e.size), "max_abs": float(e.max()), "mean_abs": float(e.mean()),
+              "max_err_over_bound": float(u.max()),
+              "within_bound": bool(over == 0 and e.mean() <= 1e-3),
+              "bound": "each |gpu - oracle| <= max(1e-2, one bf16 step), mean <= 1e-3",
+              "what": "the timed decode leg's output against the fp64 oracle on the sequences of the CPU sample"}
+    return cpu, parity
 
 
 # ----------------------------------------------------------------------------
@@ -240,7 +267,8 @@ def decode_leg(args, device, world, clocks):
     st = gqa.gqa_get_device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} after the decode leg")
-    res = {"kv_bytes": kv_bytes, "total_ms": total_max, "kernel_ms": kern_ms, "isolated_ms": res_isolated}
+    res = {"kv_bytes": kv_bytes, "total_ms": total_max, "kernel_ms": kern_ms, "isolated_ms": res_isolated,
+           "out": out.cpu()}   # the timed steps' result (every cache copy holds the same values)
 
     # end to end through the public API: pinned host inputs -> device -> decode -> host result
     qh, kh, vh, lh = (t.pin_memory() for t in (q, k, v, lens))
@@ -417,7 +445,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cpu = oracle_decode_leg(target_s=min(60.0, 5.0 + 0.2 * args.steps))
+        cpu, _ = oracle_decode_leg(target_s=min(60.0, 5.0 + 0.2 * args.steps))
         line = {"impl": "reference", "metric": metric, "value": cpu["value"], "unit": "GB/s", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16 inputs)",
@@ -503,7 +531,9 @@ def main():
                          "frac": gbs / pk["hbm"], "traffic": kernel_traffic(desc[name][1]),
                          "algorithmic_bytes_per_launch": r["kv_bytes"], "peak_source": pk["src"]}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_decode_leg(target_s=10.0)
+        line["cpu_baseline"], parity = oracle_decode_leg(target_s=10.0, gpu_out=dec["out"])
+        if parity is not None:
+            line["parity"] = parity
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
