@@ -24,3 +24,25 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Parity record of this session: every element whose error exceeded 1e-2
+    (allowed only at |oracle| >= 4, tests/_tol.py) is counted and listed."""
+    try:
+        from tests import _tol
+    except Exception:  # pragma: no cover
+        return
+    rec = _tol.RECORD
+    if not rec:
+        return
+    tr = terminalreporter
+    n_el = sum(r[1] for r in rec)
+    above = [r for r in rec if r[4]]
+    failed = [r for r in rec if r[5]]
+    tr.write_line(f"parity: {len(rec)} oracle comparisons, {n_el} outputs, worst max abs "
+                  f"{max(r[2] for r in rec):.3e}, worst mean abs {max(r[3] for r in rec):.3e}; "
+                  f"{sum(r[4] for r in above)} output(s) above 1e-2 in {len(above)} comparison(s)"
+                  + (f"; {len(failed)} comparison(s) FAILED" if failed else ""))
+    for what, n, mx, mean, a, bad in above + [r for r in failed if not r[4]]:
+        tr.write_line(f"  {'FAILED ' if bad else ''}{what}: {a} of {n} above 1e-2, max {mx:.3e}, mean {mean:.3e}")

@@ -1,8 +1,10 @@
 """8-bit (E4M3) and paged decode caches: the CUDA path through the C ABI
 against the fp64 oracle.
 
-Tolerance as for the bf16 path (tests/_tol.py): max |GPU - oracle| <= 1e-2,
-or one bf16 step where |oracle| >= 2, and mean |GPU - oracle| <= 1e-3 per call.  The oracle reads the same codes and scales,
+Tolerance as for the bf16 path (tests/_tol.py): max |GPU - oracle| <= 1e-2
+below |oracle| = 4, the derived arithmetic bound above it (with f16 weights
+for the 8-bit caches), and mean |GPU - oracle| <= 1e-3 per call.  The oracle
+reads the same codes and scales,
 so quantisation error is not part of the comparison: only the kernel's own
 rounding (Q to f16, weights to f16, fp32 sums, bf16 output) is.
 """
@@ -53,7 +55,8 @@ def status():
 def test_fp8_decode_parity(B, h, n_kv, d, lens):
     q, kc, vc, ks, vs, lens = inputs.decode_fp8_inputs(40 + h + d, B, h, n_kv, d, lens)
     got = gpu_fp8(q, kc, vc, ks, vs, lens)
-    check(got, oracle.decode_general(q, kc, vc, lens, fp8=True, k_scale=ks, v_scale=vs), "fp8 decode")
+    check(got, oracle.decode_general(q, kc, vc, lens, fp8=True, k_scale=ks, v_scale=vs), "fp8 decode", v=vc,
+          v_scale=vs, n_keys=int(lens.max()))
     for b in range(B):
         if int(lens[b]) <= 0:
             assert torch.all(got[b] == 0)
@@ -68,7 +71,8 @@ def test_fp8_decode_workloads(w):
     seed = w.seed * 1000 + w.n_kv if w.ragged else w.seed
     q, kc, vc, ks, vs, lens = inputs.decode_fp8_inputs(seed, w.B, w.h, w.n_kv, w.d, lens)
     got = gpu_fp8(q, kc, vc, ks, vs, lens)
-    check(got, oracle.decode_general(q, kc, vc, lens, fp8=True, k_scale=ks, v_scale=vs), w.name + " fp8")
+    check(got, oracle.decode_general(q, kc, vc, lens, fp8=True, k_scale=ks, v_scale=vs), w.name + " fp8", v=vc,
+          v_scale=vs, n_keys=int(lens.max()))
 
 
 def test_fp8_single_token_is_exact():
@@ -140,7 +144,8 @@ def test_paged_parity(fp8, page_size):
     got = gpu_paged(q, kp, vp, bt, lens, ks, vs)
     ref = oracle.decode_general(q, kp, vp, lens, fp8=fp8, k_scale=ks, v_scale=vs, block_table=bt,
                                 page_size=page_size)
-    check(got, ref, f"paged {'e4m3' if fp8 else 'bf16'} page {page_size}")
+    check(got, ref, f"paged {'e4m3' if fp8 else 'bf16'} page {page_size}", v=vp, v_scale=vs,
+          n_keys=int(lens.max()))
     assert torch.all(got[4] == 0)
     assert status() == _lib.GQA_OK
 
@@ -158,7 +163,7 @@ def test_paged_group_sizes(fp8, h, n_kv, d):
     kp, vp, bt = inputs.page_caches(80, k, v, lens, 32, spare_pages=2)
     got = gpu_paged(q, kp, vp, bt, lens, ks, vs)
     check(got, oracle.decode_general(q, kp, vp, lens, fp8=fp8, k_scale=ks, v_scale=vs, block_table=bt,
-                                     page_size=32), "paged group sizes")
+                                     page_size=32), "paged group sizes", v=vp, v_scale=vs, n_keys=int(lens.max()))
 
 
 @pytest.mark.parametrize("fp8", [False, True], ids=["bf16", "e4m3"])
@@ -172,7 +177,8 @@ def test_paged_workload_gqa_decode(fp8):
         ks = vs = None
     kp, vp, bt = inputs.page_caches(2, k, v, lens, 64)
     got = gpu_paged(q, kp, vp, bt, lens, ks, vs)
-    check(got, oracle.decode_general(q, k, v, lens, fp8=fp8, k_scale=ks, v_scale=vs), w.name + " paged")
+    check(got, oracle.decode_general(q, k, v, lens, fp8=fp8, k_scale=ks, v_scale=vs), w.name + " paged", v=v,
+          v_scale=vs, n_keys=int(lens.max()))
 
 
 def test_paged_bad_page_id_is_reported():
@@ -190,7 +196,8 @@ def test_paged_bad_page_id_is_reported():
     gpu_paged(q, kp, vp, bad, lens)
     assert status() == _lib.GQA_ERR_INVALID_ARG
     # sequence 0 untouched by the bad entry of sequence 1 in the first call
-    check(got[:1], oracle.decode_general(q[:1], kp, vp, lens[:1], block_table=bt[:1], page_size=64), "seq 0")
+    check(got[:1], oracle.decode_general(q[:1], kp, vp, lens[:1], block_table=bt[:1], page_size=64), "seq 0",
+          v=vp, n_keys=300)
 
 
 def test_paged_length_beyond_block_table_is_cut_and_reported():
@@ -200,7 +207,8 @@ def test_paged_length_beyond_block_table_is_cut_and_reported():
     long = torch.tensor([1000, 64], dtype=torch.int32)
     got = gpu_paged(q, kp, vp, bt, long)
     assert status() == _lib.GQA_ERR_INVALID_ARG
-    check(got, oracle.decode_general(q, kp, vp, lens, block_table=bt, page_size=64), "cut length")
+    check(got, oracle.decode_general(q, kp, vp, lens, block_table=bt, page_size=64), "cut length", v=vp,
+          n_keys=128)
 
 
 def test_device_status_clean_after_cache_tests():

@@ -61,7 +61,7 @@ def test_decode_fuzz(case):
         ref = oracle.decode(q, k, v, L)
         out = gqa.decode(*cuda(q, k, v, L))
     torch.cuda.synchronize()
-    check(out, ref, what)
+    check(out, ref, what, v=v, v_scale=vs, n_keys=max(lens))
     assert gqa.gqa_get_device_status() == _lib.GQA_OK, what
 
 
@@ -79,7 +79,7 @@ def test_prefill_fuzz(case):
     q, k, v = inputs.prefill_inputs(case, B, S_q, S_kv, h, n_kv, d)
     out = gqa.prefill(*cuda(q, k, v), causal=causal)
     torch.cuda.synchronize()
-    check(out, oracle.prefill(q, k, v, causal=causal), what)
+    check(out, oracle.prefill(q, k, v, causal=causal), what, v=v, n_keys=S_kv)
 
 
 @pytest.mark.parametrize("case", range(12))
@@ -98,7 +98,7 @@ def test_chunk_prefill_fuzz(case):
     kpd, vpd = kp.cuda(), vp.cuda()
     out = gqa.prefill_paged(q.cuda(), kn.cuda(), vn.cuda(), kpd, vpd, bt.cuda(), P.cuda())
     torch.cuda.synchronize()
-    check(out, ref, what)
+    check(out, ref, what, v=torch.cat([vn.flatten(), vp.flatten()]), n_keys=max(past) + S_q)
     bits = lambda t: t.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)   # noqa: E731
     assert np.array_equal(bits(kpd), rkp) and np.array_equal(bits(vpd), rvp), what + ": pages after the append"
 
@@ -113,5 +113,5 @@ def test_mla_fuzz(case):
     q, c, L = inputs.mla_decode_inputs(case, B, h, 512, lens)
     out = gqa.mla_decode(*cuda(q, c, L))
     torch.cuda.synchronize()
-    check(out, oracle.mla_decode(q, c, L), what)
+    check(out, oracle.mla_decode(q, c, L), what, v=c, n_keys=max(lens))
     assert gqa.gqa_get_device_status() == _lib.GQA_OK, what

@@ -25,7 +25,7 @@ def test_decode_max_batch():
     q, k, v, lens = inputs.decode_inputs(1, B, h, n_kv, d, lens)
     out = gqa.decode(q.cuda(), k.cuda(), v.cuda(), lens.cuda())
     torch.cuda.synchronize()
-    check(out, oracle.decode(q, k, v, lens), "decode B=65535")
+    check(out, oracle.decode(q, k, v, lens), "decode B=65535", v=v, n_keys=3)
     assert torch.all(out.cpu()[lens == 0] == 0)
     assert gqa.gqa_get_device_status() == _lib.GQA_OK
 
@@ -34,7 +34,7 @@ def test_decode_one_long_sequence():
     q, k, v, lens = inputs.decode_inputs(2, 1, 16, 2, 128, 131072)
     out = gqa.decode(q.cuda(), k.cuda(), v.cuda(), lens.cuda())
     torch.cuda.synchronize()
-    check(out, oracle.decode(q, k, v, lens), "decode L=131072")
+    check(out, oracle.decode(q, k, v, lens), "decode L=131072", v=v, n_keys=131072)
 
 
 def test_prefill_long_sequence_sampled():
@@ -45,14 +45,14 @@ def test_prefill_long_sequence_sampled():
     rows = [0, 1, 127, 128, 8191, 8192, 16255, 16256, 16383] + list(rng.integers(0, S, 12))
     sample = [(0, int(rng.integers(0, h)), int(r)) for r in rows]
     ref = oracle.prefill_rows(q, k, v, sample, causal=True)
-    check(torch.stack([out[b, r, i] for b, i, r in sample]), ref, "prefill S=16384")
+    check(torch.stack([out[b, r, i] for b, i, r in sample]), ref, "prefill S=16384", v=v, n_keys=S)
 
 
 def test_decode_mha_128_heads():
     q, k, v, lens = inputs.decode_inputs(4, 2, 128, 128, 128, [1000, 3])
     out = gqa.decode(q.cuda(), k.cuda(), v.cuda(), lens.cuda())
     torch.cuda.synchronize()
-    check(out, oracle.decode(q, k, v, lens), "MHA 128 heads")
+    check(out, oracle.decode(q, k, v, lens), "MHA 128 heads", v=v, n_keys=1000)
 
 
 def test_paged_decode_long_block_table():
@@ -62,5 +62,6 @@ def test_paged_decode_long_block_table():
     assert bt.shape[1] == 2048
     out = gqa.decode_paged(q.cuda(), kp.cuda(), vp.cuda(), bt.cuda(), L.cuda())
     torch.cuda.synchronize()
-    check(out, oracle.decode_general(q, kp, vp, L, block_table=bt, page_size=16), "paged 2048 pages")
+    check(out, oracle.decode_general(q, kp, vp, L, block_table=bt, page_size=16), "paged 2048 pages", v=vp,
+          n_keys=32768)
     assert gqa.gqa_get_device_status() == _lib.GQA_OK

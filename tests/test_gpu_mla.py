@@ -30,7 +30,7 @@ def run(q, c, lens, scale=None):
 def test_mla_parity(B, h, lens):
     q, c, lens = inputs.mla_decode_inputs(60 + h, B, h, 512, lens)
     got = run(q, c, lens)
-    check(got, oracle.mla_decode(q, c, lens), "MLA decode")
+    check(got, oracle.mla_decode(q, c, lens), "MLA decode", v=c, n_keys=int(lens.max()))
     for b in range(B):
         if int(lens[b]) <= 0:
             assert torch.all(got[b] == 0)
@@ -41,7 +41,7 @@ def test_mla_workload():
     """B16 h32 d_c512 L4096, every output checked."""
     w = inputs.MLA_DECODE
     q, c, lens = inputs.mla_decode_inputs(w.seed, w.B, w.h, w.d, w.kv_len)
-    check(run(q, c, lens), oracle.mla_decode(q, c, lens), w.name)
+    check(run(q, c, lens), oracle.mla_decode(q, c, lens), w.name, v=c, n_keys=w.kv_len)
 
 
 def test_mla_single_token_is_exact():
@@ -64,7 +64,7 @@ def test_mla_nan_in_previous_sequence_stays_there():
     c[99, 5] = float("nan")
     got = run(q, c, lens)
     assert torch.isnan(got[0].float()).any()
-    check(got[1:], oracle.mla_decode(q[1:], c[100:], lens[1:]), "sequence after a NaN row")
+    check(got[1:], oracle.mla_decode(q[1:], c[100:], lens[1:]), "sequence after a NaN row", v=c[100:], n_keys=30)
 
 
 def spiked_inputs(seed, B, h, lens):
@@ -83,4 +83,4 @@ def spiked_inputs(seed, B, h, lens):
 
 def test_mla_running_max_rescale():
     q, c, lens = spiked_inputs(70, 3, 32, [1000, 300, 2049])
-    check(run(q, c, lens), oracle.mla_decode(q, c, lens), "MLA with rescales")
+    check(run(q, c, lens), oracle.mla_decode(q, c, lens), "MLA with rescales", v=c, n_keys=2049)

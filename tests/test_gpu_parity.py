@@ -2,8 +2,8 @@
 
 Tolerance (bf16 inputs and outputs, fp32 accumulation): max |GPU - oracle|
 <= 1e-2 and mean |GPU - oracle| <= 1e-3 per call, the oracle being unrounded
-fp64; where |oracle| >= 2 an element may also be within one bf16 step of it
-(tests/_tol.py says why).  Index and group-mapping work is checked
+fp64; where |oracle| >= 4 (half a bf16 step is then above 1e-2) an element is
+held to the bound the arithmetic allows instead (tests/_tol.py derives it).  Index and group-mapping work is checked
 bit-exactly.
 """
 import numpy as np
@@ -44,14 +44,14 @@ def gpu_prefill(q, k, v, causal=True, scale=None):
                          ids=lambda w: w.name)
 def test_decode_workload(w):
     q, k, v, lens = inputs.workload_inputs(w)
-    check(gpu_decode(q, k, v, lens), oracle.decode(q, k, v, lens), w.name)
+    check(gpu_decode(q, k, v, lens), oracle.decode(q, k, v, lens), w.name, v=v, n_keys=int(lens.max()))
 
 
 def test_prefill_tiny_mqa():
     w = inputs.TINY_MQA_PREFILL
     q, k, v = inputs.workload_inputs(w)
     got = gpu_prefill(q, k, v, causal=True)
-    check(got, oracle.prefill(q, k, v, causal=True), w.name)
+    check(got, oracle.prefill(q, k, v, causal=True), w.name, v=v, n_keys=w.S_kv)
     # row 0 attends to key 0 alone: exactly V[0] of its group
     for i in range(w.h):
         assert torch.equal(got[0, 0, i], v[0, 0, i // w.G]), i
@@ -69,7 +69,7 @@ def test_prefill_gqa_causal_sampled():
     sample += [(w.B - 1, w.h - 1, w.S_q - 1), (0, 0, w.S_q - 1)]
     ref = oracle.prefill_rows(q, k, v, sample, causal=True)
     g = torch.stack([got[b, r, i] for b, i, r in sample])
-    check(g, ref, w.name)
+    check(g, ref, w.name, v=v, n_keys=w.S_kv)
     assert torch.isfinite(got.float()).all()
 
 
@@ -89,7 +89,8 @@ def test_prefill_gqa_causal_sampled():
 ])
 def test_prefill_shapes(B, S_q, S_kv, h, n_kv, d, causal):
     q, k, v = inputs.prefill_inputs(100 + S_q, B, S_q, S_kv, h, n_kv, d)
-    check(gpu_prefill(q, k, v, causal=causal), oracle.prefill(q, k, v, causal=causal), "prefill")
+    check(gpu_prefill(q, k, v, causal=causal), oracle.prefill(q, k, v, causal=causal), "prefill", v=v,
+          n_keys=S_kv)
 
 
 @pytest.mark.parametrize("G", [1, 3, 8, 12, 16, 24, 32, 48, 64, 128])
@@ -99,7 +100,7 @@ def test_decode_group_sizes(G, d):
     lens = torch.tensor([0, 1, 63, 64, 65, 130, 1000, 17], dtype=torch.int32)
     q, k, v, lens = inputs.decode_inputs(G * 7 + d, len(lens), G * n_kv, n_kv, d, lens)
     got = gpu_decode(q, k, v, lens)
-    check(got, oracle.decode(q, k, v, lens), f"decode G={G} d={d}")
+    check(got, oracle.decode(q, k, v, lens), f"decode G={G} d={d}", v=v, n_keys=int(lens.max()))
     assert torch.all(got[0] == 0)           # zero-length sequence -> zero row
 
 
@@ -131,19 +132,21 @@ def test_group_mapping_bit_exact():
 
 def test_zero_scale_is_mean_of_v():
     q, k, v, lens = inputs.decode_inputs(8, 2, 8, 2, 128, torch.tensor([700, 5], dtype=torch.int32))
-    check(gpu_decode(q, k, v, lens, scale=0.0), oracle.decode(q, k, v, lens, scale=0.0), "scale 0 decode")
+    check(gpu_decode(q, k, v, lens, scale=0.0), oracle.decode(q, k, v, lens, scale=0.0), "scale 0 decode", v=v,
+          n_keys=int(lens.max()))
     q, k, v = inputs.prefill_inputs(8, 1, 150, 150, 4, 2, 64)
-    check(gpu_prefill(q, k, v, scale=0.0), oracle.prefill(q, k, v, scale=0.0), "scale 0 prefill")
+    check(gpu_prefill(q, k, v, scale=0.0), oracle.prefill(q, k, v, scale=0.0), "scale 0 prefill", v=v, n_keys=150)
 
 
 def test_large_scores_stay_finite():
     """Scores far from 0 exercise the running-max rescaling."""
     q, k, v = inputs.prefill_inputs(9, 1, 300, 300, 2, 1, 128)
     q = (q.float() * 4).to(torch.bfloat16)
-    check(gpu_prefill(q, k, v, causal=True), oracle.prefill(q, k, v, causal=True), "large scores prefill")
+    check(gpu_prefill(q, k, v, causal=True), oracle.prefill(q, k, v, causal=True), "large scores prefill", v=v,
+          n_keys=300)
     q2, k2, v2, lens = inputs.decode_inputs(9, 2, 8, 1, 128, 900)
     q2 = (q2.float() * 4).to(torch.bfloat16)
-    check(gpu_decode(q2, k2, v2, lens), oracle.decode(q2, k2, v2, lens), "large scores decode")
+    check(gpu_decode(q2, k2, v2, lens), oracle.decode(q2, k2, v2, lens), "large scores decode", v=v2, n_keys=900)
 
 
 def test_split_count_does_not_change_the_result():
@@ -191,3 +194,36 @@ def test_repeatable():
 
 def test_device_status_clean():
     assert gqa.gqa_get_device_status() == 0
+
+
+def test_lengths_past_the_cache_rows_are_cut_and_reported():
+    """The binding passes the caches' row count (gqa_decode_rows): a sequence whose
+    rows would run past the caches is cut to the rows that exist, reported, and
+    nothing past the caches is read."""
+    q, k, v, lens = inputs.decode_inputs(15, 3, 16, 2, 128, torch.tensor([600, 600, 50], dtype=torch.int32))
+    k, v = k[:1000].contiguous(), v[:1000].contiguous()          # the caches hold 1000 of the 1250 rows
+    assert gqa.gqa_get_device_status() == 0
+    got = gpu_decode(q, k, v, lens)
+    assert gqa.gqa_get_device_status() == 1                      # GQA_ERR_INVALID_ARG
+    cut = torch.tensor([600, 400, 0], dtype=torch.int32)         # sequence 2 starts past the rows: empty
+    check(got, oracle.decode(q, k, v, cut), "cut at the cache rows", v=v, n_keys=600)
+    assert torch.all(got[2] == 0)
+    # the same lengths over caches that hold every row: clean
+    q, k, v, lens = inputs.decode_inputs(15, 3, 16, 2, 128, torch.tensor([600, 600, 50], dtype=torch.int32))
+    gpu_decode(q, k, v, lens)
+    assert gqa.gqa_get_device_status() == 0
+
+
+def test_mla_and_fp8_lengths_past_the_cache_rows_are_cut_and_reported():
+    q, c, lens = inputs.mla_decode_inputs(16, 2, 32, 512, [300, 300])
+    c = c[:450].contiguous()
+    got = gqa.mla_decode(q.cuda(), c.cuda(), lens.cuda()).cpu()
+    assert gqa.gqa_get_device_status() == 1
+    check(got, oracle.mla_decode(q, c, torch.tensor([300, 150], dtype=torch.int32)), "MLA cut", v=c, n_keys=300)
+    q, kc, vc, ks, vs, lens = inputs.decode_fp8_inputs(17, 2, 8, 2, 128, [300, 300])
+    kc, vc = kc[:450].contiguous(), vc[:450].contiguous()
+    got = gqa.decode_fp8(q.cuda(), kc.cuda(), vc.cuda(), ks.cuda(), vs.cuda(), lens.cuda()).cpu()
+    assert gqa.gqa_get_device_status() == 1
+    ref = oracle.decode_general(q, kc, vc, torch.tensor([300, 150], dtype=torch.int32), fp8=True, k_scale=ks,
+                                v_scale=vs)
+    check(got, ref, "E4M3 cut", v=vc, v_scale=vs, n_keys=300)
