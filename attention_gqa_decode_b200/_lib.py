@@ -14,15 +14,18 @@ _handle = None
 GQA_OK, GQA_ERR_INVALID_ARG, GQA_ERR_UNSUPPORTED, GQA_ERR_CUDA, GQA_ERR_TIMEOUT = range(5)
 
 # every entry point include/gqa.h declares, with its ctypes signature
-_vp, _i, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+_vp, _i, _f, _i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64
 SIGNATURES = {
     "gqa_prefill": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
+    "gqa_decode_rows": ([_vp, _vp, _vp, _i64, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
+    "gqa_decode_fp8_rows": ([_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_paged": ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_paged_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_prefill_paged": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_mla_decode": ([_vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp], _i),
+    "gqa_mla_decode_rows": ([_vp, _vp, _i64, _vp, _vp, _i, _i, _i, _f, _vp], _i),
     "gqa_status_string": ([_i], ctypes.c_char_p),
     "gqa_get_device_status": ([_vp], _i),
 }
@@ -38,20 +41,25 @@ def library_path() -> str:
     return _LIB_PATH
 
 
+def load_library(path: str) -> ctypes.CDLL:
+    """A CDLL of a build of the library at `path` with every declared signature set."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m attention_gqa_decode_b200.build` (nvcc, sm_100a)")
+    h = ctypes.CDLL(path)
+    for name, (args, res) in SIGNATURES.items():
+        fn = getattr(h, name)
+        fn.argtypes = args
+        fn.restype = res
+    return h
+
+
 def lib() -> ctypes.CDLL:
     """The loaded CUDA library; raises if it has not been built."""
     global _handle
     with _lock:
         if _handle is None:
-            if not os.path.exists(_LIB_PATH):
-                raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
-                                   "`python -m attention_gqa_decode_b200.build` (nvcc, sm_100a)")
-            h = ctypes.CDLL(_LIB_PATH)
-            for name, (args, res) in SIGNATURES.items():
-                fn = getattr(h, name)
-                fn.argtypes = args
-                fn.restype = res
-            _handle = h
+            _handle = load_library(_LIB_PATH)
     return _handle
 
 
@@ -73,6 +81,21 @@ def gqa_prefill(q, k, v, out, B, S_q, S_kv, h, n_kv, d_h, causal, scale, stream)
 
 def gqa_decode(q, k_cache, v_cache, seqlens, out, B, h, n_kv, d_h, scale, stream) -> int:
     return lib().gqa_decode(q, k_cache, v_cache, seqlens, out, B, h, n_kv, d_h, float(scale), stream)
+
+
+def gqa_decode_rows(q, k_cache, v_cache, cache_rows, seqlens, out, B, h, n_kv, d_h, scale, stream) -> int:
+    return lib().gqa_decode_rows(q, k_cache, v_cache, int(cache_rows), seqlens, out, B, h, n_kv, d_h, float(scale),
+                                 stream)
+
+
+def gqa_decode_fp8_rows(q, k_cache, v_cache, cache_rows, k_scale, v_scale, seqlens, out, B, h, n_kv, d_h, scale,
+                        stream) -> int:
+    return lib().gqa_decode_fp8_rows(q, k_cache, v_cache, int(cache_rows), k_scale, v_scale, seqlens, out, B, h, n_kv,
+                                     d_h, float(scale), stream)
+
+
+def gqa_mla_decode_rows(q_absorbed, c_kv, cache_rows, seqlens, out, B, h, d_c, scale, stream) -> int:
+    return lib().gqa_mla_decode_rows(q_absorbed, c_kv, int(cache_rows), seqlens, out, B, h, d_c, float(scale), stream)
 
 
 def gqa_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, B, h, n_kv, d_h, scale, stream) -> int:
@@ -151,9 +174,11 @@ def prefill(q, k, v, causal: bool = True, scale: float | None = None, out=None, 
 
 
 def decode(q, k_cache, v_cache, seqlens, scale: float | None = None, out=None, stream=None):
-    """One decode step: q [B,h,d], packed caches [sum(seqlens),n_kv,d], seqlens int32 [B] (CUDA).
+    """One decode step: q [B,h,d], packed caches [T,n_kv,d], seqlens int32 [B] (CUDA).
 
-    Returns out [B,h,d].  Sequence b's tokens start at cache row sum(seqlens[:b]).
+    Returns out [B,h,d].  Sequence b's tokens start at cache row sum(seqlens[:b]);
+    a sequence that would end past row T is cut there and GQA_ERR_INVALID_ARG is
+    recorded in the device status word (gqa_get_device_status).
     """
     import torch
     _check(q, "q", 3), _check(k_cache, "k_cache", 3), _check(v_cache, "v_cache", 3)
@@ -173,10 +198,10 @@ def decode(q, k_cache, v_cache, seqlens, scale: float | None = None, out=None, s
         if out.shape != q.shape:
             raise ValueError("out must have q's shape")
     with torch.cuda.device(q.device):
-        st = gqa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(), out.data_ptr(),
-                        B, h, n_kv, d, scale, _stream_ptr(stream))
+        st = gqa_decode_rows(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), T, seqlens.data_ptr(),
+                             out.data_ptr(), B, h, n_kv, d, scale, _stream_ptr(stream))
     if st != GQA_OK:
-        raise GQAError(st, "gqa_decode")
+        raise GQAError(st, "gqa_decode_rows")
     return out
 
 
@@ -236,11 +261,11 @@ def decode_fp8(q, k_cache, v_cache, k_scale, v_scale, seqlens, scale: float | No
         if out.shape != q.shape:
             raise ValueError("out must have q's shape")
     with torch.cuda.device(q.device):
-        st = gqa_decode_fp8(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), k_scale.data_ptr(),
-                            v_scale.data_ptr(), seqlens.data_ptr(), out.data_ptr(), B, h, n_kv, d, scale,
-                            _stream_ptr(stream))
+        st = gqa_decode_fp8_rows(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), T, k_scale.data_ptr(),
+                                 v_scale.data_ptr(), seqlens.data_ptr(), out.data_ptr(), B, h, n_kv, d, scale,
+                                 _stream_ptr(stream))
     if st != GQA_OK:
-        raise GQAError(st, "gqa_decode_fp8")
+        raise GQAError(st, "gqa_decode_fp8_rows")
     return out
 
 
@@ -352,8 +377,8 @@ def mla_decode(q_absorbed, c_kv, seqlens, scale: float | None = None, out=None, 
         if out.shape != q_absorbed.shape:
             raise ValueError("out must have q_absorbed's shape")
     with torch.cuda.device(q_absorbed.device):
-        st = gqa_mla_decode(q_absorbed.data_ptr(), c_kv.data_ptr(), seqlens.data_ptr(), out.data_ptr(), B, h, d_c,
-                            scale, _stream_ptr(stream))
+        st = gqa_mla_decode_rows(q_absorbed.data_ptr(), c_kv.data_ptr(), c_kv.shape[0], seqlens.data_ptr(),
+                                 out.data_ptr(), B, h, d_c, scale, _stream_ptr(stream))
     if st != GQA_OK:
-        raise GQAError(st, "gqa_mla_decode")
+        raise GQAError(st, "gqa_mla_decode_rows")
     return out

@@ -8,21 +8,30 @@
 #include "common.cuh"
 
 namespace gqa {
-__device__ int g_status = 0;   // see gqa_get_device_status()
+__device__ int g_status = 0;         // see gqa_get_device_status()
+__device__ int g_status_taken = 0;   // the value the last status read exchanged out of g_status
+#ifdef GQA_WAIT_TEST
+__device__ int g_test_stall = 0;     // wait-test build: producers leave their first stage unloaded
+#endif
+
+// Exchange the status word for 0 in one atomic step, so that an error a kernel
+// records concurrently is either returned now or kept for the next read.
+__global__ void take_status_kernel() { g_status_taken = atomicExch(&g_status, 0); }
 
 int launch_prefill(const void *q, const void *k, const void *v, void *out, int B, int S_q, int S_kv, int h, int n_kv,
                    int d, int causal, float scale, cudaStream_t stream);
 int launch_decode(const void *q, const void *k, const void *v, const int32_t *seqlens, void *out, int B, int h,
-                  int n_kv, int d, float scale, cudaStream_t stream);
+                  int n_kv, int d, float scale, long long cache_rows, cudaStream_t stream);
 int launch_prefill_paged(const void *q, const void *k_new, const void *v_new, void *k_pages, void *v_pages,
                          const int32_t *block_table, int max_blocks, int page_size, int num_pages,
                          const int32_t *past_lens, void *out, int B, int S_q, int h, int n_kv, int d, float scale,
                          cudaStream_t stream);
 int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h, float scale,
-                      cudaStream_t stream);
+                      long long cache_rows, cudaStream_t stream);
 int launch_decode_ex(const void *q, const void *k, const void *v, const float *k_scale, const float *v_scale,
                      const int32_t *seqlens, const int32_t *block_table, int max_blocks, int page_size,
-                     int num_pages, void *out, int B, int h, int n_kv, int d, float scale, cudaStream_t stream);
+                     int num_pages, void *out, int B, int h, int n_kv, int d, float scale, long long cache_rows,
+                     cudaStream_t stream);
 }  // namespace gqa
 
 namespace gqa_host {
@@ -80,6 +89,22 @@ int *device_status() {
     return ptrs[dev];
 }
 
+#ifdef GQA_WAIT_TEST
+int *device_test_stall() {
+    static int *ptrs[64] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, gqa::g_test_stall) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int *>(p);
+    }
+    return ptrs[dev];
+}
+#endif
+
 int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -92,6 +117,13 @@ int sm_count() {
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 static bool scale_ok(float s) { return std::isfinite(s) && s >= 0.f; }
+
+// The token extent the packed-cache entry points without a row count give
+// their tensor maps: the caller's contract covers the rows, and offsets past
+// it are cut and reported by the kernels.
+constexpr long long kOpenRows = 1LL << 30;
+
+static bool rows_ok(int64_t rows) { return rows >= 0 && rows <= 0x7FFFFFFFLL; }
 
 extern "C" {
 
@@ -107,8 +139,9 @@ int gqa_prefill(const void *q, const void *k, const void *v, void *out, int B, i
     return gqa::launch_prefill(q, k, v, out, B, S_q, S_kv, h, n_kv, d_h, causal, scale, stream);
 }
 
-int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens, void *out, int B,
-               int h, int n_kv, int d_h, float scale, cudaStream_t stream) {
+static int decode_bf16(const void *q, const void *k_cache, const void *v_cache, long long cache_rows,
+                       const int32_t *seqlens, void *out, int B, int h, int n_kv, int d_h, float scale,
+                       cudaStream_t stream) {
     if (!q || !k_cache || !v_cache || !seqlens || !out) return GQA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(seqlens) & 3u))
@@ -117,7 +150,19 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const in
     if (!scale_ok(scale)) return GQA_ERR_INVALID_ARG;
     if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
     if (static_cast<long>(n_kv) * ((h / n_kv + 63) / 64) > 65535) return GQA_ERR_UNSUPPORTED;
-    return gqa::launch_decode(q, k_cache, v_cache, seqlens, out, B, h, n_kv, d_h, scale, stream);
+    return gqa::launch_decode(q, k_cache, v_cache, seqlens, out, B, h, n_kv, d_h, scale, cache_rows, stream);
+}
+
+int gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens, void *out, int B,
+               int h, int n_kv, int d_h, float scale, cudaStream_t stream) {
+    return decode_bf16(q, k_cache, v_cache, kOpenRows, seqlens, out, B, h, n_kv, d_h, scale, stream);
+}
+
+int gqa_decode_rows(const void *q, const void *k_cache, const void *v_cache, int64_t cache_rows,
+                    const int32_t *seqlens, void *out, int B, int h, int n_kv, int d_h, float scale,
+                    cudaStream_t stream) {
+    if (!rows_ok(cache_rows)) return GQA_ERR_INVALID_ARG;
+    return decode_bf16(q, k_cache, v_cache, cache_rows, seqlens, out, B, h, n_kv, d_h, scale, stream);
 }
 
 // Checks shared by every decode entry point (cache pointers are checked by the caller).
@@ -159,7 +204,19 @@ int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, cons
     if (st == GQA_OK) st = decode_args_ok(q, seqlens, out, B, h, n_kv, d_h, scale);
     if (st != GQA_OK) return st;
     return gqa::launch_decode_ex(q, k_cache, v_cache, k_scale, v_scale, seqlens, nullptr, 0, 0, 0, out, B, h, n_kv,
-                                 d_h, scale, stream);
+                                 d_h, scale, kOpenRows, stream);
+}
+
+int gqa_decode_fp8_rows(const void *q, const void *k_cache, const void *v_cache, int64_t cache_rows,
+                        const float *k_scale, const float *v_scale, const int32_t *seqlens, void *out, int B, int h,
+                        int n_kv, int d_h, float scale, cudaStream_t stream) {
+    if (!rows_ok(cache_rows)) return GQA_ERR_INVALID_ARG;
+    int st = caches_ok(k_cache, v_cache);
+    if (st == GQA_OK) st = scales_ok(k_scale, v_scale);
+    if (st == GQA_OK) st = decode_args_ok(q, seqlens, out, B, h, n_kv, d_h, scale);
+    if (st != GQA_OK) return st;
+    return gqa::launch_decode_ex(q, k_cache, v_cache, k_scale, v_scale, seqlens, nullptr, 0, 0, 0, out, B, h, n_kv,
+                                 d_h, scale, cache_rows, stream);
 }
 
 int gqa_decode_paged(const void *q, const void *k_pages, const void *v_pages, const int32_t *block_table,
@@ -170,7 +227,7 @@ int gqa_decode_paged(const void *q, const void *k_pages, const void *v_pages, co
     if (st == GQA_OK) st = decode_args_ok(q, seqlens, out, B, h, n_kv, d_h, scale);
     if (st != GQA_OK) return st;
     return gqa::launch_decode_ex(q, k_pages, v_pages, nullptr, nullptr, seqlens, block_table, max_blocks, page_size,
-                                 num_pages, out, B, h, n_kv, d_h, scale, stream);
+                                 num_pages, out, B, h, n_kv, d_h, scale, kOpenRows, stream);
 }
 
 int gqa_decode_paged_fp8(const void *q, const void *k_pages, const void *v_pages, const float *k_scale,
@@ -183,7 +240,7 @@ int gqa_decode_paged_fp8(const void *q, const void *k_pages, const void *v_pages
     if (st == GQA_OK) st = decode_args_ok(q, seqlens, out, B, h, n_kv, d_h, scale);
     if (st != GQA_OK) return st;
     return gqa::launch_decode_ex(q, k_pages, v_pages, k_scale, v_scale, seqlens, block_table, max_blocks, page_size,
-                                 num_pages, out, B, h, n_kv, d_h, scale, stream);
+                                 num_pages, out, B, h, n_kv, d_h, scale, kOpenRows, stream);
 }
 
 int gqa_prefill_paged(const void *q, const void *k_new, const void *v_new, void *k_pages, void *v_pages,
@@ -205,15 +262,26 @@ int gqa_prefill_paged(const void *q, const void *k_new, const void *v_new, void 
                                      num_pages, past_lens, out, B, S_q, h, n_kv, d_h, scale, stream);
 }
 
-int gqa_mla_decode(const void *q_absorbed, const void *c_kv, const int32_t *seqlens, void *out, int B, int h,
-                   int d_c, float scale, cudaStream_t stream) {
+static int mla_decode(const void *q_absorbed, const void *c_kv, long long cache_rows, const int32_t *seqlens,
+                      void *out, int B, int h, int d_c, float scale, cudaStream_t stream) {
     if (!q_absorbed || !c_kv || !seqlens || !out) return GQA_ERR_INVALID_ARG;
     if (!aligned16(q_absorbed) || !aligned16(c_kv) || !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
         return GQA_ERR_INVALID_ARG;
     if (B <= 0 || B > 65535 || h <= 0 || h > 65535 * 16) return GQA_ERR_INVALID_ARG;
     if (!scale_ok(scale)) return GQA_ERR_INVALID_ARG;
     if (d_c != 512) return GQA_ERR_UNSUPPORTED;
-    return gqa::launch_mla_decode(q_absorbed, c_kv, seqlens, out, B, h, scale, stream);
+    return gqa::launch_mla_decode(q_absorbed, c_kv, seqlens, out, B, h, scale, cache_rows, stream);
+}
+
+int gqa_mla_decode(const void *q_absorbed, const void *c_kv, const int32_t *seqlens, void *out, int B, int h,
+                   int d_c, float scale, cudaStream_t stream) {
+    return mla_decode(q_absorbed, c_kv, kOpenRows, seqlens, out, B, h, d_c, scale, stream);
+}
+
+int gqa_mla_decode_rows(const void *q_absorbed, const void *c_kv, int64_t cache_rows, const int32_t *seqlens,
+                        void *out, int B, int h, int d_c, float scale, cudaStream_t stream) {
+    if (!rows_ok(cache_rows)) return GQA_ERR_INVALID_ARG;
+    return mla_decode(q_absorbed, c_kv, cache_rows, seqlens, out, B, h, d_c, scale, stream);
 }
 
 const char *gqa_status_string(int status) {
@@ -228,11 +296,24 @@ const char *gqa_status_string(int status) {
 }
 
 int gqa_get_device_status(cudaStream_t stream) {
+    // one reader at a time per process: the exchanged value passes through g_status_taken
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    gqa::take_status_kernel<<<1, 1, 0, stream>>>();
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, gqa::g_status_taken, sizeof(int), 0, cudaMemcpyDeviceToHost, stream) !=
+        cudaSuccess)
+        return GQA_ERR_CUDA;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return GQA_ERR_CUDA;
-    int v = 0, zero = 0;
-    if (cudaMemcpyFromSymbol(&v, gqa::g_status, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
-    if (cudaMemcpyToSymbol(gqa::g_status, &zero, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
     return v;
 }
+
+#ifdef GQA_WAIT_TEST
+int gqa_test_set_stall(int on) {
+    const int v = on ? 1 : 0;
+    return cudaMemcpyToSymbol(gqa::g_test_stall, &v, sizeof(int)) == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+#endif
 
 }  // extern "C"

@@ -23,7 +23,19 @@ constexpr int kStatusInvalid = 1;   // == GQA_ERR_INVALID_ARG (a bad value found
 constexpr int kStatusTimeout = 4;   // == GQA_ERR_TIMEOUT
 
 // A wait gives up after this many nanoseconds of global time (about a second).
+// The wait-test build (GQA_WAIT_TEST, a separate library only the tests load)
+// gives up after a millisecond, and its producers leave their first stage
+// unloaded while the library's test stall word is non-zero, so that a test
+// can make a bounded wait run out and see the kernel return an error status.
+#ifdef GQA_WAIT_TEST
+constexpr unsigned long long kWaitLimitNs = 1000000ull;
+#define GQA_TEST_STALL_FIELD const int *stall;   // the test stall word (wait-test build only)
+#define GQA_STALLED(prm) (*reinterpret_cast<const volatile int *>((prm).stall) != 0)
+#else
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+#define GQA_TEST_STALL_FIELD
+#define GQA_STALLED(prm) false
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -432,6 +444,20 @@ bool once_per_device(std::atomic<unsigned long long> &done, int dev, F &&set) {
 
 // Device address of the library's status word on the current device (null on failure).
 int *device_status();
+
+#ifdef GQA_WAIT_TEST
+// Device address of the test stall word on the current device (wait-test build only).
+int *device_test_stall();
+#define GQA_SET_TEST_STALL(prm)                         \
+    do {                                                \
+        (prm).stall = gqa_host::device_test_stall();    \
+        if (!(prm).stall) return 3;                     \
+    } while (0)
+#else
+#define GQA_SET_TEST_STALL(prm) \
+    do {                        \
+    } while (0)
+#endif
 
 
 }  // namespace gqa_host

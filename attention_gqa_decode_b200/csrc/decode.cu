@@ -103,8 +103,10 @@ struct DecodeParams {
     const int32_t *block_table;       // paged caches: [B, max_blocks]
     int max_blocks, page_size, num_pages;
     int B, h, n_kv, G, slices;        // slices = ceil(G / kDecMaxHeads)
+    long long cache_rows;             // packed caches: rows the caches hold (the tensor maps' extent)
     float scale_log2;                 // scale * log2(e), >= 0
     int *status;                      // the library's device status word
+    GQA_TEST_STALL_FIELD
 };
 
 template <int D, KvFmt F, int STAGES, bool TR>
@@ -384,7 +386,7 @@ __global__ void __launch_bounds__(kDecThreads, MINB)
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::kRingBytes);
     uint64_t *empty = full + STAGES;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + STAGES);
-    int *red = reinterpret_cast<int *>(empty + STAGES) + 1;   // [kDecWarps + 1] partial sums
+    long long *red = reinterpret_cast<long long *>(empty + STAGES + 1);   // [kDecWarps + 1] partial sums
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = gridDim.x, split = blockIdx.x;
@@ -407,22 +409,28 @@ __global__ void __launch_bounds__(kDecThreads, MINB)
         tma_prefetch_desc(&tm_v);
     }
 
-    // packed caches: first cache row of sequence b = sum of the earlier (non-negative) lengths
-    int acc = 0;
+    // packed caches: first cache row of sequence b = sum of the earlier (non-negative) lengths (64-bit)
+    long long acc = 0;
     if (!PAGED)
         for (int i = threadIdx.x; i < b; i += kDecThreads) acc += max(p.seqlens[i], 0);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) red[warp] = acc;
     __syncthreads();
-    int off = 0;
+    long long off64 = 0;
 #pragma unroll
-    for (int w = 0; w <= kDecWarps; ++w) off += red[w];
+    for (int w = 0; w <= kDecWarps; ++w) off64 += red[w];
     int L = max(p.seqlens[b], 0);
     if (PAGED && L > p.max_blocks * p.page_size) {   // longer than its block-table row
         if (threadIdx.x == 0) record_status(p.status, kStatusInvalid);
         L = p.max_blocks * p.page_size;
     }
+    if (!PAGED && off64 + L > p.cache_rows) {   // the lengths ask for rows the caches do not hold
+        if (threadIdx.x == 0) record_status(p.status, kStatusInvalid);
+        L = static_cast<int>(max(0LL, p.cache_rows - off64));
+    }
+    // off + L <= cache_rows <= INT32_MAX whenever a row is read (the host bounds cache_rows)
+    const int off = static_cast<int>(min(off64, p.cache_rows));
 
     // this split's stages: stage i covers tokens [t0, min(t0 + TOK, L)), t0 = TOK * (first + i)
     const int n_total = (L + TOK - 1) / TOK;
@@ -452,11 +460,16 @@ __global__ void __launch_bounds__(kDecThreads, MINB)
         int ids = (PAGED && n_stages > 0) ? batch_of(0) : 0;
         int ids_next = (PAGED && n_stages * pieces > 32) ? batch_of(1) : 0;
         int issued = 0;
+        const int first_loaded = GQA_STALLED(p) ? 1 : 0;   // wait-test build: stage 0 never arrives
         for (int i = 0; i < n_stages; ++i) {
             const int slot = i % STAGES, use = i / STAGES;
             int ok = 1;
             if (lane == 0 && use > 0) ok = mbar_wait(&empty[slot], (use - 1) & 1, abort_flag, p.status);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (i < first_loaded) {
+                ++issued;
+                continue;
+            }
             const int t0 = (first + i) * TOK;
             uint8_t *kdst = smem + slot * SM::kStageBytes;
             uint8_t *vdst = kdst + SM::kTileBytes;
@@ -498,7 +511,7 @@ __global__ void __launch_bounds__(kDecThreads, MINB)
             ++issued;
         }
         if (lane == 0 && *abort_flag) {   // let the copies in flight land before the CTA moves on
-            for (int i = max(0, issued - STAGES); i < issued; ++i)
+            for (int i = max(first_loaded, issued - STAGES); i < issued; ++i)
                 mbar_wait_drain(&full[i % STAGES], (i / STAGES) & 1, p.status);
         }
         __syncwarp();
@@ -871,6 +884,7 @@ struct DecodeCall {
     const int32_t *seqlens, *block_table;
     void *out;
     int B, h, n_kv, max_blocks, page_size, num_pages;
+    long long cache_rows;   // packed caches: rows the caches hold (0 < rows <= INT32_MAX, or open: 2^30)
     float scale;
     cudaStream_t stream;
 };
@@ -894,8 +908,10 @@ static int launch_decode_t(const DecodeCall &c) {
     const CUtensorMapSwizzle swz = Geo::kRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap tk, tv;
     if (!PAGED) {
-        // [tokens, n_kv, D]; the token extent is left open (the caller owns the lengths)
-        const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(c.n_kv), 1ull << 30};
+        // [tokens, n_kv, D]; the token extent is the caches' row count (the kernel cuts
+        // lengths that ask for more rows and reports them)
+        const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(c.n_kv),
+                                  static_cast<uint64_t>(std::max(c.cache_rows, 1LL))};
         const uint64_t strides[2] = {D * E, static_cast<uint64_t>(c.n_kv) * D * E};
         const uint32_t box[3] = {static_cast<uint32_t>(Geo::kBoxInner), 1, static_cast<uint32_t>(Geo::kTok)};
         if (!gqa_host::encode_tensor_map_ex(&tk, dt, swz, c.k, 3, dims, strides, box)) return 3;
@@ -938,9 +954,11 @@ static int launch_decode_t(const DecodeCall &c) {
     prm.n_kv = c.n_kv;
     prm.G = G;
     prm.slices = slices;
+    prm.cache_rows = c.cache_rows;
     prm.scale_log2 = c.scale * 1.4426950408889634f;
     prm.status = gqa_host::device_status();
     if (!prm.status) return 3;
+    GQA_SET_TEST_STALL(prm);
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(P, c.n_kv * slices, c.B);
@@ -975,16 +993,18 @@ static int launch_decode_f(const DecodeCall &c, int d) {
 }
 
 int launch_decode(const void *q, const void *k, const void *v, const int32_t *seqlens, void *out, int B, int h,
-                  int n_kv, int d, float scale, cudaStream_t stream) {
-    const DecodeCall c{q, k, v, nullptr, nullptr, seqlens, nullptr, out, B, h, n_kv, 0, 0, 0, scale, stream};
+                  int n_kv, int d, float scale, long long cache_rows, cudaStream_t stream) {
+    const DecodeCall c{q, k, v, nullptr, nullptr, seqlens, nullptr, out, B, h, n_kv, 0, 0, 0, cache_rows, scale,
+                       stream};
     return launch_decode_f<KvFmt::kBf16, false>(c, d);
 }
 
 int launch_decode_ex(const void *q, const void *k, const void *v, const float *k_scale, const float *v_scale,
                      const int32_t *seqlens, const int32_t *block_table, int max_blocks, int page_size,
-                     int num_pages, void *out, int B, int h, int n_kv, int d, float scale, cudaStream_t stream) {
+                     int num_pages, void *out, int B, int h, int n_kv, int d, float scale, long long cache_rows,
+                     cudaStream_t stream) {
     const DecodeCall c{q,   k,         v,         k_scale, v_scale, seqlens, block_table, out,  B,
-                       h,   n_kv,      max_blocks, page_size, num_pages, scale, stream};
+                       h,   n_kv,      max_blocks, page_size, num_pages, cache_rows, scale, stream};
     const bool fp8 = k_scale != nullptr, paged = block_table != nullptr;
     if (fp8 && paged) return launch_decode_f<KvFmt::kE4m3, true>(c, d);
     if (fp8) return launch_decode_f<KvFmt::kE4m3, false>(c, d);

@@ -50,8 +50,10 @@ struct MlaParams {
     const int32_t *seqlens;
     __nv_bfloat16 *out;
     int B, h, groups;              // groups = ceil(h / 16)
+    long long cache_rows;          // rows the latent cache holds (the tensor map's extent)
     float scale_log2;              // scale * log2(e), >= 0
     int *status;
+    GQA_TEST_STALL_FIELD
 };
 
 struct MlaSmem {
@@ -77,7 +79,7 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
     uint64_t *sfull = empty + kMlaStages;          // all partial scores of a stage written
     uint64_t *sfree = sfull + 1;                   // all partial scores of a stage read
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sfree + 1);
-    int *red = reinterpret_cast<int *>(sfree + 1) + 1;   // [kMlaWarps + 1]
+    long long *red = reinterpret_cast<long long *>(sfree + 2);   // [kMlaWarps + 1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int P = gridDim.x, split = blockIdx.x;
@@ -97,17 +99,23 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
     }
     if (warp == kMlaWarps && lane == 0) tma_prefetch_desc(&tm_c);
 
-    // first cache row of sequence b
-    int acc = 0;
+    // first cache row of sequence b (64-bit sum of the earlier non-negative lengths)
+    long long acc = 0;
     for (int i = threadIdx.x; i < b; i += kMlaThreads) acc += max(p.seqlens[i], 0);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) red[warp] = acc;
     __syncthreads();
-    int off = 0;
+    long long off64 = 0;
 #pragma unroll
-    for (int w = 0; w <= kMlaWarps; ++w) off += red[w];
-    const int L = max(p.seqlens[b], 0);
+    for (int w = 0; w <= kMlaWarps; ++w) off64 += red[w];
+    int L = max(p.seqlens[b], 0);
+    if (off64 + L > p.cache_rows) {   // the lengths ask for rows the cache does not hold
+        if (threadIdx.x == 0) record_status(p.status, kStatusInvalid);
+        L = static_cast<int>(max(0LL, p.cache_rows - off64));
+    }
+    // off + L <= cache_rows <= INT32_MAX whenever a row is read (the host bounds cache_rows)
+    const int off = static_cast<int>(min(off64, p.cache_rows));
     const int n_total = (L + kMlaTok - 1) / kMlaTok;
     const int per_split = (n_total + P - 1) / P;
     const int first = split * per_split;
@@ -117,9 +125,14 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int issued = 0;
+            const int first_loaded = GQA_STALLED(p) ? 1 : 0;   // wait-test build: stage 0 never arrives
             for (int i = 0; i < n_stages; ++i) {
                 const int slot = i % kMlaStages, use = i / kMlaStages;
                 if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, abort_flag, p.status)) break;
+                if (i < first_loaded) {
+                    ++issued;
+                    continue;
+                }
                 const int t0 = (first + i) * kMlaTok;
                 // the last stage is shifted back to end at the sequence end (never past the cache)
                 const int z = off + min(t0, L - kMlaTok);
@@ -131,7 +144,7 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
                 ++issued;
             }
             if (*abort_flag) {
-                for (int i = max(0, issued - kMlaStages); i < issued; ++i)
+                for (int i = max(first_loaded, issued - kMlaStages); i < issued; ++i)
                     mbar_wait_drain(&full[i % kMlaStages], (i / kMlaStages) & 1, p.status);
             }
         }
@@ -397,7 +410,7 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
 // host launcher
 
 int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h, float scale,
-                      cudaStream_t stream) {
+                      long long cache_rows, cudaStream_t stream) {
     auto kern = gqa_mla_decode_kernel;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 3;
@@ -408,7 +421,8 @@ int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, v
         }))
         return 3;
     CUtensorMap tc;
-    const uint64_t dims[2] = {static_cast<uint64_t>(kMlaDc), 1ull << 30};   // token extent left open
+    // token extent = the cache's rows (the kernel cuts lengths that ask for more and reports them)
+    const uint64_t dims[2] = {static_cast<uint64_t>(kMlaDc), static_cast<uint64_t>(std::max(cache_rows, 1LL))};
     const uint64_t strides[1] = {static_cast<uint64_t>(kMlaDc) * 2};
     const uint32_t box[2] = {64, kMlaTok};
     if (!gqa_host::encode_tensor_map(&tc, c_kv, 2, dims, strides, box)) return 3;
@@ -424,9 +438,11 @@ int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, v
     prm.B = B;
     prm.h = h;
     prm.groups = groups;
+    prm.cache_rows = cache_rows;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.status = gqa_host::device_status();
     if (!prm.status) return 3;
+    GQA_SET_TEST_STALL(prm);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(P, groups, B);
     cfg.blockDim = dim3(kMlaThreads, 1, 1);

@@ -71,6 +71,7 @@ struct PrefillParams {
     const __nv_bfloat16 *k_new, *v_new;
     __nv_bfloat16 *k_pages, *v_pages;
     int max_blocks, page_size, num_pages;
+    GQA_TEST_STALL_FIELD
 };
 
 template <int D>
@@ -206,6 +207,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             int ids_next = (PAGED && n_past * pieces > 32) ? batch_of(1) : 0;
             int item = 0;
             bool stop = false;
+            const int first_loaded = GQA_STALLED(p) ? 1 : 0;   // wait-test build: K tile 0 never arrives
             for (int j = 0; j < nmax && !stop; ++j) {
                 for (int kv = 0; kv < 2; ++kv, ++item) {
                     const int slot = item % kPfRing, use = item / kPfRing;
@@ -215,6 +217,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         stop = true;
                         break;
                     }
+                    if (item < first_loaded) continue;
                     uint8_t *dst = sRing + slot * SM::kTile;
                     if (PAGED && j < n_past) {
                         // rows [0, valid) of this tile are cached tokens: one box per page piece
@@ -248,7 +251,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
             if (lane == 0 && *abort_flag) {   // let the copies in flight land before TMEM and smem go away
                 mbar_wait_drain(qfull, 0, p.status);
-                for (int i = max(0, item - kPfRing); i < item; ++i)
+                for (int i = max(first_loaded, item - kPfRing); i < item; ++i)
                     mbar_wait_drain(&full[i % kPfRing], (i / kPfRing) & 1, p.status);
             }
             __syncwarp();
@@ -558,6 +561,7 @@ static int launch_prefill_t(const PrefillCall &c) {
     prm.scale_log2 = c.scale * 1.4426950408889634f;
     prm.status = gqa_host::device_status();
     if (!prm.status) return 3;
+    GQA_SET_TEST_STALL(prm);
     prm.block_table = c.block_table;
     prm.past_lens = c.past_lens;
     prm.k_new = static_cast<const __nv_bfloat16 *>(c.k);

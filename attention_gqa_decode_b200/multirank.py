@@ -17,6 +17,20 @@ def shard_range(n: int, rank: int, world: int) -> tuple[int, int]:
     return lo, lo + base + (1 if rank < extra else 0)
 
 
+def packed_shard(seqlens, rank: int, world: int) -> tuple[int, int, int, int]:
+    """This rank's share of a decode batch whose caches are packed.
+
+    Returns (lo, hi, row_lo, row_hi): sequences [lo, hi) of the batch
+    (shard_range), whose cached tokens are rows [row_lo, row_hi) of the packed
+    caches -- sequence b starts at the sum of the earlier non-negative lengths.
+    The shard is itself a packed batch: q[lo:hi], caches[row_lo:row_hi],
+    seqlens[lo:hi]."""
+    lens = [max(int(x), 0) for x in seqlens]
+    lo, hi = shard_range(len(lens), rank, world)
+    row_lo = sum(lens[:lo])
+    return lo, hi, row_lo, row_lo + sum(lens[lo:hi])
+
+
 def max_over_ranks(x: float, device=None) -> float:
     """The maximum of x over all ranks (x itself without a process group)."""
     import torch

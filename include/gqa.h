@@ -93,13 +93,31 @@ int gqa_prefill(const void *q, const void *k, const void *v, void *out,
  * Query head i of sequence b attends to all seqlens[b] tokens of KV head
  * i / (h / n_kv).  A length <= 0 produces a zero row (counted as zero rows
  * of the packed caches).  The caches must hold at least sum(max(seqlens, 0))
- * rows; the library cannot check this (the lengths live on the device).
+ * rows: this entry point has no row count to check against (the lengths live
+ * on the device), so it only cuts and reports a sequence that would end past
+ * row 2^30; gqa_decode_rows checks the actual row count.
  * Errors: as gqa_prefill (B, h, n_kv <= 0, h % n_kv != 0, pointers, scale,
  * d_h), plus GQA_ERR_INVALID_ARG for B > 65535.
  */
 int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
                const int32_t *seqlens, void *out,
                int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
+
+/*
+ * gqa_decode with the caches' row count: the same computation, over packed
+ * caches that hold `cache_rows` rows ([cache_rows, n_kv, d_h] each).  The
+ * lengths live on the device, so the host cannot compare them with the
+ * caches; here the kernel does.  A sequence whose rows would end past
+ * cache_rows (its first row is the sum of the earlier non-negative lengths,
+ * summed in 64 bits) is cut to the rows that exist, and GQA_ERR_INVALID_ARG
+ * is recorded in the device status word (gqa_get_device_status); no row past
+ * cache_rows is ever read.  The Python binding calls this form.
+ * Errors: as gqa_decode, plus GQA_ERR_INVALID_ARG for cache_rows < 0 or
+ * cache_rows > INT32_MAX (tile coordinates are 32-bit).
+ */
+int gqa_decode_rows(const void *q, const void *k_cache, const void *v_cache, int64_t cache_rows,
+                    const int32_t *seqlens, void *out,
+                    int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
 
 /*
  * Decode over an 8-bit cache ("Multi-Query Attention (MQA)" (inferensys
@@ -126,6 +144,13 @@ int gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache,
                    const float *k_scale, const float *v_scale,
                    const int32_t *seqlens, void *out,
                    int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
+
+/* gqa_decode_fp8 over packed E4M3 caches of `cache_rows` rows, with the row
+ * check of gqa_decode_rows (lengths past the caches cut and reported). */
+int gqa_decode_fp8_rows(const void *q, const void *k_cache, const void *v_cache, int64_t cache_rows,
+                        const float *k_scale, const float *v_scale,
+                        const int32_t *seqlens, void *out,
+                        int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
 
 /*
  * Decode over a paged bf16 cache ("Multi-Query Attention (MQA)" (inferensys
@@ -215,16 +240,30 @@ int gqa_prefill_paged(const void *q, const void *k_new, const void *v_new,
 int gqa_mla_decode(const void *q_absorbed, const void *c_kv, const int32_t *seqlens, void *out,
                    int B, int h, int d_c, float scale, cudaStream_t stream);
 
+/* gqa_mla_decode over a latent cache of `cache_rows` rows, with the row check
+ * of gqa_decode_rows (lengths past the cache cut and reported). */
+int gqa_mla_decode_rows(const void *q_absorbed, const void *c_kv, int64_t cache_rows,
+                        const int32_t *seqlens, void *out,
+                        int B, int h, int d_c, float scale, cudaStream_t stream);
+
 /* A static, human-readable name for a gqa_status_t value. */
 const char *gqa_status_string(int status);
 
 /*
- * Synchronises `stream`, then returns and clears the library's device status
- * word for the current device: GQA_OK, GQA_ERR_TIMEOUT if a kernel gave up
- * on an internal wait since the last call, or GQA_ERR_INVALID_ARG if a kernel
- * met a bad value that lives on the device (a page id, a length beyond the
- * block table, a negative or non-finite cache scale).  The first error wins.  Returns GQA_ERR_CUDA if the
- * synchronisation itself fails.
+ * Returns and clears the library's device status word for the current
+ * device: GQA_OK, GQA_ERR_TIMEOUT if a kernel gave up on an internal wait
+ * since the last read, or GQA_ERR_INVALID_ARG if a kernel met a bad value
+ * that lives on the device (a page id, a length beyond the block table or
+ * the caches, a negative or non-finite cache scale).  The first error
+ * recorded since the last read wins.
+ * The word is per DEVICE, not per stream: it collects what every kernel of
+ * this library on the device recorded, whatever its stream.  The read is
+ * enqueued on `stream` as one atomic exchange (the word is swapped for 0),
+ * then `stream` is synchronised; an error that a kernel on another stream
+ * records meanwhile is never lost -- it is returned by this read or by the
+ * next.  To attribute an error to one call, synchronise the device (or every
+ * stream that runs this library's kernels) before the call and read the word
+ * after it.  Returns GQA_ERR_CUDA if the read or the synchronisation fails.
  */
 int gqa_get_device_status(cudaStream_t stream);
 

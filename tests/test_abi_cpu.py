@@ -160,3 +160,39 @@ def test_prefill_paged_rejects(L, args, expect):
 ])
 def test_mla_decode_rejects(L, args, expect):
     assert gqa.gqa_mla_decode(*args, None) == expect
+
+
+@pytest.mark.parametrize("rows,expect", [
+    (-1, _lib.GQA_ERR_INVALID_ARG),                # negative row count
+    ((1 << 31), _lib.GQA_ERR_INVALID_ARG),         # above INT32_MAX (tile coordinates are 32-bit)
+])
+def test_row_checked_entry_points_reject_bad_row_counts(L, rows, expect):
+    assert gqa.gqa_decode_rows(A, A, A, rows, A, A, 2, 4, 2, 128, 0.1, None) == expect
+    assert gqa.gqa_decode_fp8_rows(A, A, A, rows, A, A, A, A, 2, 4, 2, 128, 0.1, None) == expect
+    assert gqa.gqa_mla_decode_rows(A, A, rows, A, A, 2, 32, 512, 0.04, None) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    # the argument checks of the forms without a row count apply too
+    ((0, A, A, 100, A, A, 2, 4, 2, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, 100, A, A, 2, 4, 3, 128, 0.1), _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, A, 100, A, A, 2, 4, 2, 32, 0.1), _lib.GQA_ERR_UNSUPPORTED),
+])
+def test_decode_rows_rejects(L, args, expect):
+    assert gqa.gqa_decode_rows(*args, None) == expect
+
+
+def test_wait_test_library_exports_everything():
+    """libgqa_b200_waittest.so: every entry point of gqa.h plus the one of gqa_waittest.h."""
+    from attention_gqa_decode_b200.build import WAITTEST_LIB
+    build()
+    text = open(os.path.join(ROOT, "include", "gqa_waittest.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    extra = re.findall(r"^\s*int\s+(gqa_\w+)\s*\(", text, flags=re.M)
+    assert extra == ["gqa_test_set_stall"]
+    W = _lib.load_library(WAITTEST_LIB)
+    for name in declared_functions() + extra:
+        assert isinstance(getattr(W, name), ctypes._CFuncPtr), name
+    # the product library has no test hook
+    with pytest.raises(AttributeError):
+        getattr(gqa.lib(), "gqa_test_set_stall")
