@@ -72,6 +72,12 @@ namespace gqa {
 constexpr int kDecWarps = 4;       // consumer warps
 constexpr int kDecThreads = (kDecWarps + 1) * 32;
 constexpr int kDecMaxHeads = 64;   // query heads one CTA serves (4 m-tiles of 16)
+// bf16 caches: the softmax weights reach the tensor cores as bf16.  For a
+// sequence of at most this many tokens, where a few keys can carry most of a
+// row's weight (and the weights' rounding does not average out), they also
+// go as the bf16 remainder p - bf16(p) in a second product, so they are
+// carried to about 16 bits.
+constexpr int kSplitAllBelow = 256;
 
 enum class KvFmt { kBf16, kE4m3 };
 
@@ -192,6 +198,7 @@ __device__ __forceinline__ void consume_transposed(const DecodeParams &p, uint8_
             continue;
         }
         const bool partial = row_lo > tw0 || row_hi < tw0 + TWARP;
+        const bool split = !FP8 && L <= kSplitAllBelow;   // warp-uniform
         const uint32_t kbase = smem_u32(smem + slot * SM::kStageBytes) + tw0 * RB;
         const uint32_t vbase = kbase + SM::kTileBytes;
 
@@ -259,7 +266,7 @@ __device__ __forceinline__ void consume_transposed(const DecodeParams &p, uint8_
             o[mt][3] *= alpha[1];
         }
         // P^T B fragments: pack a row (token) of two heads, transpose the 8x8 blocks
-        uint32_t pb[TT][2];
+        uint32_t pb[TT][2], pr[TT][2];   // the weights (bf16) and, on split stages, their bf16 remainders
         float2 ls = make_float2(0.f, 0.f);
 #pragma unroll
         for (int tt = 0; tt < TT; ++tt) {
@@ -280,7 +287,14 @@ __device__ __forceinline__ void consume_transposed(const DecodeParams &p, uint8_
             } else {
                 lo = pack_bf16x2(e0, e1);
                 hi = pack_bf16x2(e2, e3);
-                ls = fadd2(ls, fadd2(unpack_bf16x2(lo), unpack_bf16x2(hi)));
+                const float2 ul = unpack_bf16x2(lo), uh = unpack_bf16x2(hi);
+                ls = fadd2(ls, fadd2(ul, uh));
+                if (split) {   // remainders (exact in fp32), rounded to bf16 for the second product
+                    const uint32_t rl = pack_bf16x2(e0 - ul.x, e1 - ul.y), rh = pack_bf16x2(e2 - uh.x, e3 - uh.y);
+                    ls = fadd2(ls, fadd2(unpack_bf16x2(rl), unpack_bf16x2(rh)));
+                    pr[tt][0] = movmatrix_trans(rl);
+                    pr[tt][1] = movmatrix_trans(rh);
+                }
             }
             pb[tt][0] = movmatrix_trans(lo);   // P[head g8][tokens 2 q4, 2 q4 + 1]
             pb[tt][1] = movmatrix_trans(hi);   // P[head g8][tokens 2 q4 + 8, 2 q4 + 9]
@@ -316,6 +330,7 @@ __device__ __forceinline__ void consume_transposed(const DecodeParams &p, uint8_
                         a[3] &= mhi;
                     }
                     mma_bf16_16816(o[mt], a, pb[tt][0], pb[tt][1]);
+                    if (split) mma_bf16_16816(o[mt], a, pr[tt][0], pr[tt][1]);
                 }
             } else {
                 const uint32_t rowaddr = vbase + (tt * 16 + arow) * RB;
@@ -586,6 +601,7 @@ __global__ void __launch_bounds__(kDecThreads, MINB)
                 const int tw0 = ti * TWARP + pass * TPW;              // first row of this pass
                 if (row_lo >= tw0 + TPW || row_hi <= tw0) continue;  // no valid row here
                 const bool partial = row_lo > tw0 || row_hi < tw0 + TPW;
+                const bool split = !FP8 && L <= kSplitAllBelow;   // warp-uniform
                 const uint32_t kbase = stage + tw0 * RB;
                 const uint32_t vbase = kbase + SM::kTileBytes;
 
@@ -658,7 +674,7 @@ __global__ void __launch_bounds__(kDecThreads, MINB)
                     o[nt][3] *= alpha[1];
                 }
                 // P as bf16 (f16 for 8-bit caches) A fragments; the running sums add the rounded weights
-                uint32_t pa[KKS][4];
+                uint32_t pa[KKS][4], par[KKS][4];   // the weights and, on split stages, their bf16 remainders
                 float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int nt = 0; nt < NTS; ++nt) {
@@ -685,8 +701,17 @@ __global__ void __launch_bounds__(kDecThreads, MINB)
                     } else {
                         lo = pack_bf16x2(e0, e1);
                         hi = pack_bf16x2(e2, e3);
-                        ls0 = fadd2(ls0, unpack_bf16x2(lo));
-                        ls1 = fadd2(ls1, unpack_bf16x2(hi));
+                        const float2 ul = unpack_bf16x2(lo), uh = unpack_bf16x2(hi);
+                        ls0 = fadd2(ls0, ul);
+                        ls1 = fadd2(ls1, uh);
+                        if (split) {   // remainders (exact in fp32), rounded to bf16 for the second product
+                            const uint32_t rl = pack_bf16x2(e0 - ul.x, e1 - ul.y);
+                            const uint32_t rh = pack_bf16x2(e2 - uh.x, e3 - uh.y);
+                            ls0 = fadd2(ls0, unpack_bf16x2(rl));
+                            ls1 = fadd2(ls1, unpack_bf16x2(rh));
+                            par[nt >> 1][(nt & 1) * 2 + 0] = rl;
+                            par[nt >> 1][(nt & 1) * 2 + 1] = rh;
+                        }
                     }
                     pa[nt >> 1][(nt & 1) * 2 + 0] = lo;
                     pa[nt >> 1][(nt & 1) * 2 + 1] = hi;
@@ -723,6 +748,10 @@ __global__ void __launch_bounds__(kDecThreads, MINB)
                             }
                             mma_bf16_16816(o[2 * dp], pa[kk], b0, b1);
                             mma_bf16_16816(o[2 * dp + 1], pa[kk], b2, b3);
+                            if (split) {
+                                mma_bf16_16816(o[2 * dp], par[kk], b0, b1);
+                                mma_bf16_16816(o[2 * dp + 1], par[kk], b2, b3);
+                            }
                         }
                     } else {
 #pragma unroll

@@ -44,6 +44,10 @@ constexpr int kMlaPanelBytes = kMlaTok * 128;
 constexpr int kMlaStageBytes = kMlaPanels * kMlaPanelBytes;   // 32 KB
 constexpr int kMlaMaxSplit = 8;
 constexpr float kMlaRescale = 8.0f;               // lazy rescale threshold (log2 units)
+// The softmax weights reach the tensor cores as bf16.  For a sequence of at
+// most this many tokens, where a few keys can carry most of a row's weight,
+// they also go as the bf16 remainder p - bf16(p) in a second product.
+constexpr int kMlaSplitAllBelow = 256;
 
 struct MlaParams {
     const __nv_bfloat16 *q;
@@ -291,7 +295,8 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
                     o[nt][3] *= alpha[1];
                 }
             }
-            uint32_t pa[KKS][4];
+            const bool split = L <= kMlaSplitAllBelow;   // warp-uniform
+            uint32_t pa[KKS][4], par[KKS][4];   // the weights and, on split stages, their bf16 remainders
             float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int nt = 0; nt < NTS; ++nt) {
@@ -306,8 +311,16 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
                 const uint32_t lo = pack_bf16x2(e0, e1), hi = pack_bf16x2(e2, e3);
                 pa[nt >> 1][(nt & 1) * 2 + 0] = lo;
                 pa[nt >> 1][(nt & 1) * 2 + 1] = hi;
-                ls0 = fadd2(ls0, unpack_bf16x2(lo));
-                ls1 = fadd2(ls1, unpack_bf16x2(hi));
+                const float2 ul = unpack_bf16x2(lo), uh = unpack_bf16x2(hi);
+                ls0 = fadd2(ls0, ul);
+                ls1 = fadd2(ls1, uh);
+                if (split) {   // remainders (exact in fp32), rounded to bf16 for the second product
+                    const uint32_t rl = pack_bf16x2(e0 - ul.x, e1 - ul.y), rh = pack_bf16x2(e2 - uh.x, e3 - uh.y);
+                    par[nt >> 1][(nt & 1) * 2 + 0] = rl;
+                    par[nt >> 1][(nt & 1) * 2 + 1] = rh;
+                    ls0 = fadd2(ls0, unpack_bf16x2(rl));
+                    ls1 = fadd2(ls1, unpack_bf16x2(rh));
+                }
             }
             l_run[0] += ls0.x + ls0.y;
             l_run[1] += ls1.x + ls1.y;
@@ -329,6 +342,10 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
                                                           (((chunk & 7) ^ (lane & 7)) << 4));
                     mma_bf16_16816(o[2 * dp], pa[kk], b0 & mlo, b1 & mhi);
                     mma_bf16_16816(o[2 * dp + 1], pa[kk], b2 & mlo, b3 & mhi);
+                    if (split) {
+                        mma_bf16_16816(o[2 * dp], par[kk], b0 & mlo, b1 & mhi);
+                        mma_bf16_16816(o[2 * dp + 1], par[kk], b2 & mlo, b3 & mhi);
+                    }
                 }
             }
             __syncwarp();

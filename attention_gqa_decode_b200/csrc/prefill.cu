@@ -60,6 +60,13 @@ constexpr int kPfThreads = 384;  // softmax warpgroups 0 and 1; warpgroup 2 = pr
 constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 80;
 static_assert(256 * kRegsSoftmax + 128 * kRegsOther <= kPfThreads * 168, "register split exceeds the launch");
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+// The softmax weights reach the tensor cores as bf16 (written over S in
+// TMEM).  For a query tile whose first row sees at most this many keys --
+// rows where a few keys can carry most of the weight and the weights'
+// rounding does not average out -- the bf16 remainders p - bf16(p) are also
+// written (over the upper half of S) and multiplied by V in a second product,
+// so those weights are carried to about 16 bits.
+constexpr int kPfSplitKeys = 256;
 
 struct PrefillParams {
     __nv_bfloat16 *out;
@@ -96,6 +103,15 @@ __device__ __forceinline__ int kv_tiles_for(int rows_begin, int S_q, int S_kv, i
 __device__ __forceinline__ int chunk_tiles_for(int rows_begin, int S_q, int n_past) {
     if (rows_begin >= S_q) return 0;
     return n_past + min(rows_begin + kPfRows - 1, S_q - 1) / kPfKeys + 1;
+}
+
+// Whether the weights of the query tile starting at row `row0` go to the
+// tensor cores with their bf16 remainders: its first row (the one that sees
+// the fewest keys) sees at most kPfSplitKeys keys.
+template <bool PAGED>
+__device__ __forceinline__ bool split_weights(const PrefillParams &p, int row0, int past) {
+    const int keys = PAGED ? past + row0 + 1 : p.causal ? min(p.S_kv, row0 + (p.S_kv - p.S_q) + 1) : p.S_kv;
+    return keys <= kPfSplitKeys;
 }
 
 template <int D, bool PAGED>
@@ -277,15 +293,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         umma_ss(d_tmem, sdesc_sw128(a0 + o, 16, 1024), sdesc_sw128(b0 + o, 16, 1024), idesc_qk, ks > 0);
                     }
                 };
-                auto issue_pv = [&](int t, int item, bool acc) {
+                // rem: the second product, A = the weights' bf16 remainders (upper half of S)
+                auto issue_pv = [&](int t, int item, bool acc, bool rem) {
                     const uint32_t d_tmem = tmem + 256 + t * D;
-                    const uint32_t a_tmem = tmem + t * 128;
+                    const uint32_t a_tmem = tmem + t * 128 + (rem ? kPfKeys / 2 : 0);
                     const uint32_t b0 = ring_base + (item % kPfRing) * SM::kTile;
     #pragma unroll
                     for (int kk = 0; kk < kPfKeys / 16; ++kk)
                         umma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, SM::kHalf, 1024), idesc_pv,
-                                (acc || kk > 0) ? 1u : 0u);
+                                (acc || rem || kk > 0) ? 1u : 0u);
                 };
+                const bool split_t[2] = {split_weights<PAGED>(p, q0, past), split_weights<PAGED>(p, q0 + kPfRows, past)};
                 bool ok = mbar_wait(qfull, 0, abort_flag, p.status) && ready(0);
                 if (ok) {
                     if (n_t0 > 0) { issue_qk(0, 0); umma_commit(&sfull[0]); }
@@ -315,7 +333,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                 fence_proxy_async_smem();   // generic-proxy stores before the tensor core reads
                             }
                         }
-                        issue_pv(t, 2 * j + 1, j > 0);
+#pragma unroll 1
+                        for (int ps = 0; ps < (split_t[t] ? 2 : 1); ++ps) issue_pv(t, 2 * j + 1, j > 0, ps > 0);
                         if (j + 1 < n_t) {
                             if (!k_next) {
                                 if (!ready(2 * j + 2)) { ok = false; continue; }
@@ -371,6 +390,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint32_t tS = tmem + t * 128 + lane_off;
         const uint32_t tO = tmem + 256 + t * D + lane_off;
         const float cl2 = p.scale_log2;
+        const bool split = split_weights<PAGED>(p, q0 + t * kPfRows, past);   // warpgroup-uniform
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_t; ++j) {
@@ -431,23 +451,43 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     m_used = m_new;
                 }
             }
-            // P = exp2(S * scale * log2(e) - m) as packed bf16, written back over S;
+            // P = exp2(S * scale * log2(e) - m) as packed bf16, written back over S
+            // (and, for a split tile, the bf16 remainders over the upper half of S);
             // the running sum adds exactly the rounded weights P V uses
             float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            // the weights of a key pair (masked keys add nothing, also when scale == 0)
+            auto weights = [&](int c) -> float2 {
+                const float2 x = ffma2_bcast(__uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)), cl2, -m_used);
+                float2 w = make_float2(exp2f(x.x), exp2f(x.y));
+                if (masked) {
+                    if (c > lim_c) w.x = 0.f;
+                    if (c + 1 > lim_c) w.y = 0.f;
+                }
+                return w;
+            };
+            if (split) {   // the remainders w - bf16(w), exact in fp32, rounded to bf16 (computed first: the main pass below
+                           // then consumes the S registers as it goes)
+#pragma unroll
+                for (int ch = 0; ch < kPfKeys / 32; ++ch) {
+                    uint32_t rk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float2 w = weights(ch * 32 + 2 * e);
+                        const float2 u = unpack_bf16x2(pack_bf16x2(w.x, w.y));
+                        rk[e] = pack_bf16x2(w.x - u.x, w.y - u.y);
+                        rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(rk[e]));
+                    }
+                    tmem_st16(tS + kPfKeys / 2 + ch * 16, rk);
+                }
+            }
 #pragma unroll
             for (int ch = 0; ch < kPfKeys / 32; ++ch) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const int c = ch * 32 + 2 * e;
-                    const float2 x = ffma2_bcast(__uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)), cl2, -m_used);
-                    uint32_t pp = pack_bf16x2(exp2f(x.x), exp2f(x.y));
-                    if (masked) {   // masked keys add nothing (also when scale == 0)
-                        if (c > lim_c) pp &= 0xFFFF0000u;
-                        if (c + 1 > lim_c) pp &= 0x0000FFFFu;
-                    }
-                    pk[e] = pp;
-                    rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(pp));
+                    const float2 w = weights(ch * 32 + 2 * e);
+                    pk[e] = pack_bf16x2(w.x, w.y);
+                    rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(pk[e]));
                 }
                 tmem_st16(tS + ch * 16, pk);
             }
