@@ -19,6 +19,9 @@ SIGNATURES = {
     "gqa_prefill": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_rows": ([_vp, _vp, _vp, _i64, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
+    "gqa_decode_split": ([_vp, _vp, _vp, _i64, _vp, _vp, _i, _i, _i, _i, _f, _vp, ctypes.c_size_t, _vp], _i),
+    "gqa_decode_split_workspace_bytes": ([_i, _i, _i, _i], ctypes.c_size_t),
+    "gqa_decode_split_counter_bytes": ([_i, _i, _i], ctypes.c_size_t),
     "gqa_decode_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_fp8_rows": ([_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_paged": ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
@@ -86,6 +89,20 @@ def gqa_decode(q, k_cache, v_cache, seqlens, out, B, h, n_kv, d_h, scale, stream
 def gqa_decode_rows(q, k_cache, v_cache, cache_rows, seqlens, out, B, h, n_kv, d_h, scale, stream) -> int:
     return lib().gqa_decode_rows(q, k_cache, v_cache, int(cache_rows), seqlens, out, B, h, n_kv, d_h, float(scale),
                                  stream)
+
+
+def gqa_decode_split(q, k_cache, v_cache, cache_rows, seqlens, out, B, h, n_kv, d_h, scale, workspace,
+                     workspace_bytes, stream) -> int:
+    return lib().gqa_decode_split(q, k_cache, v_cache, int(cache_rows), seqlens, out, B, h, n_kv, d_h, float(scale),
+                                  workspace, int(workspace_bytes), stream)
+
+
+def gqa_decode_split_workspace_bytes(B, h, n_kv, d_h) -> int:
+    return int(lib().gqa_decode_split_workspace_bytes(B, h, n_kv, d_h))
+
+
+def gqa_decode_split_counter_bytes(B, h, n_kv) -> int:
+    return int(lib().gqa_decode_split_counter_bytes(B, h, n_kv))
 
 
 def gqa_decode_fp8_rows(q, k_cache, v_cache, cache_rows, k_scale, v_scale, seqlens, out, B, h, n_kv, d_h, scale,
@@ -173,13 +190,79 @@ def prefill(q, k, v, causal: bool = True, scale: float | None = None, out=None, 
     return out
 
 
+# Groups of at least this many query heads per KV head, over caches holding at
+# least SPLIT_MIN_MEAN_ROWS rows per sequence, go to the split-KV tensor-core
+# kernel (gqa_decode_split); everything else to the cluster kernel.
+SPLIT_MIN_GROUP = 32
+SPLIT_MIN_MEAN_ROWS = 256
+_workspaces = {}   # device index -> [workspace tensor, bytes at its start known to be zero after the last call]
+
+
+def split_workspace(device, nbytes: int, counter_bytes: int):
+    """A device workspace of at least nbytes for gqa_decode_split whose first
+    counter_bytes are zero: one per device, kept and grown as needed (every call
+    leaves its counters zero; a call with more counters than the earlier ones gets
+    the extra bytes zeroed first).  Calls that share it must not overlap on the GPU.
+    Make the first call of a shape before capturing a CUDA graph that uses it."""
+    import torch
+    dev = torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    ent = _workspaces.get(key)
+    if ent is None or ent[0].numel() < nbytes:
+        ent = [torch.zeros(max(nbytes, 1), dtype=torch.uint8, device=torch.device("cuda", key)), nbytes]
+        _workspaces[key] = ent
+    if counter_bytes > ent[1]:
+        ent[0][ent[1]:counter_bytes].zero_()
+    ent[1] = counter_bytes   # after the call only its own counters are known zero (the rest is scratch)
+    return ent[0]
+
+
+def decode_split(q, k_cache, v_cache, seqlens, scale: float | None = None, out=None, stream=None, workspace=None):
+    """gqa_decode_split: the decode step with the batch's tokens divided evenly among
+    the SMs (tensor-core products, partial results merged in a workspace).  Same
+    arguments and result as :func:`decode`; ``workspace`` defaults to the binding's
+    per-device workspace (:func:`split_workspace`)."""
+    import torch
+    _check(q, "q", 3), _check(k_cache, "k_cache", 3), _check(v_cache, "v_cache", 3)
+    B, h, d = q.shape
+    T, n_kv, dk = k_cache.shape
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or dk != d:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k_cache.shape)} v{tuple(v_cache.shape)}")
+    _check_seqlens(seqlens, B)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check(out, "out", 3)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    with torch.cuda.device(q.device):
+        need = gqa_decode_split_workspace_bytes(B, h, n_kv, d)
+        ws = workspace if workspace is not None else \
+            split_workspace(q.device, need, gqa_decode_split_counter_bytes(B, h, n_kv))
+        st = gqa_decode_split(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), T, seqlens.data_ptr(),
+                              out.data_ptr(), B, h, n_kv, d, scale, ws.data_ptr(), ws.numel() * ws.element_size(),
+                              _stream_ptr(stream))
+    if st != GQA_OK:
+        raise GQAError(st, "gqa_decode_split")
+    return out
+
+
 def decode(q, k_cache, v_cache, seqlens, scale: float | None = None, out=None, stream=None):
     """One decode step: q [B,h,d], packed caches [T,n_kv,d], seqlens int32 [B] (CUDA).
 
     Returns out [B,h,d].  Sequence b's tokens start at cache row sum(seqlens[:b]);
     a sequence that would end past row T is cut there and GQA_ERR_INVALID_ARG is
-    recorded in the device status word (gqa_get_device_status).
+    recorded in the device status word (gqa_get_device_status).  Groups of
+    SPLIT_MIN_GROUP or more query heads per KV head over caches of at least
+    SPLIT_MIN_MEAN_ROWS rows per sequence run on gqa_decode_split, the rest on
+    gqa_decode_rows (the lengths stay on the device; the choice uses the shapes).
     """
+    if q.dim() == 3 and k_cache.dim() == 3 and k_cache.shape[1] > 0 and \
+            q.shape[1] // max(k_cache.shape[1], 1) >= SPLIT_MIN_GROUP and \
+            k_cache.shape[0] >= SPLIT_MIN_MEAN_ROWS * q.shape[0]:
+        return decode_split(q, k_cache, v_cache, seqlens, scale=scale, out=out, stream=stream)
     import torch
     _check(q, "q", 3), _check(k_cache, "k_cache", 3), _check(v_cache, "v_cache", 3)
     B, h, d = q.shape

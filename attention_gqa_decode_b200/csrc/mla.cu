@@ -27,6 +27,8 @@
 
 #include <algorithm>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace cg = cooperative_groups;
@@ -210,6 +212,11 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
         float s[NTS][4];
         bool ok = n_stages == 0 || landed(0);
         if (ok && n_stages > 0) partial_scores(stage_addr(0), s);
+        // the stage loop, compiled twice: with the weights' bf16 remainders (sequences of at
+        // most kMlaSplitAllBelow tokens) and without, so the long-sequence path carries no
+        // extra registers
+        auto stage_loop = [&](auto split_tag) {
+            constexpr bool kSplit = decltype(split_tag)::value;
         for (int i = 0; i < n_stages && ok; ++i) {
             const int slot = i % kMlaStages;
             const int t0 = (first + i) * kMlaTok;
@@ -295,7 +302,7 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
                     o[nt][3] *= alpha[1];
                 }
             }
-            const bool split = L <= kMlaSplitAllBelow;   // warp-uniform
+            constexpr bool split = kSplit;
             uint32_t pa[KKS][4], par[KKS][4];   // the weights and, on split stages, their bf16 remainders
             float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -314,7 +321,7 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
                 const float2 ul = unpack_bf16x2(lo), uh = unpack_bf16x2(hi);
                 ls0 = fadd2(ls0, ul);
                 ls1 = fadd2(ls1, uh);
-                if (split) {   // remainders (exact in fp32), rounded to bf16 for the second product
+                if constexpr (split) {   // remainders (exact in fp32), rounded to bf16 for the second product
                     const uint32_t rl = pack_bf16x2(e0 - ul.x, e1 - ul.y), rh = pack_bf16x2(e2 - uh.x, e3 - uh.y);
                     par[nt >> 1][(nt & 1) * 2 + 0] = rl;
                     par[nt >> 1][(nt & 1) * 2 + 1] = rh;
@@ -342,7 +349,7 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
                                                           (((chunk & 7) ^ (lane & 7)) << 4));
                     mma_bf16_16816(o[2 * dp], pa[kk], b0 & mlo, b1 & mhi);
                     mma_bf16_16816(o[2 * dp + 1], pa[kk], b2 & mlo, b3 & mhi);
-                    if (split) {
+                    if constexpr (split) {
                         mma_bf16_16816(o[2 * dp], par[kk], b0 & mlo, b1 & mhi);
                         mma_bf16_16816(o[2 * dp + 1], par[kk], b2 & mlo, b3 & mhi);
                     }
@@ -358,6 +365,11 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
                 s[nt][3] = sn[nt][3];
             }
         }
+        };
+        if (L <= kMlaSplitAllBelow)
+            stage_loop(std::true_type{});
+        else
+            stage_loop(std::false_type{});
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);

@@ -44,6 +44,7 @@
 // warps attend.  The attention never reads a slot that is being written:
 // past tiles only cover positions < past.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -112,6 +113,16 @@ template <bool PAGED>
 __device__ __forceinline__ bool split_weights(const PrefillParams &p, int row0, int past) {
     const int keys = PAGED ? past + row0 + 1 : p.causal ? min(p.S_kv, row0 + (p.S_kv - p.S_q) + 1) : p.S_kv;
     return keys <= kPfSplitKeys;
+}
+
+// The second P V product of a split tile (A = the weights' bf16 remainders in
+// TMEM, B = V): out of line, so the common path of the 80-register MMA issuer
+// keeps its registers.
+__device__ __noinline__ void pf_issue_pv_rem(uint32_t d_tmem, uint32_t a_tmem, uint32_t b0, uint32_t lbo,
+                                             uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < kPfKeys / 16; ++kk)
+        umma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, lbo, 1024), idesc, 1u);
 }
 
 template <int D, bool PAGED>
@@ -293,23 +304,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         umma_ss(d_tmem, sdesc_sw128(a0 + o, 16, 1024), sdesc_sw128(b0 + o, 16, 1024), idesc_qk, ks > 0);
                     }
                 };
-                // rem: the second product, A = the weights' bf16 remainders (upper half of S)
-                auto issue_pv = [&](int t, int item, bool acc, bool rem) {
+                auto issue_pv = [&](int t, int item, bool acc) {
                     const uint32_t d_tmem = tmem + 256 + t * D;
-                    const uint32_t a_tmem = tmem + t * 128 + (rem ? kPfKeys / 2 : 0);
+                    const uint32_t a_tmem = tmem + t * 128;
                     const uint32_t b0 = ring_base + (item % kPfRing) * SM::kTile;
     #pragma unroll
                     for (int kk = 0; kk < kPfKeys / 16; ++kk)
                         umma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, SM::kHalf, 1024), idesc_pv,
-                                (acc || rem || kk > 0) ? 1u : 0u);
+                                (acc || kk > 0) ? 1u : 0u);
                 };
-                const bool split_t[2] = {split_weights<PAGED>(p, q0, past), split_weights<PAGED>(p, q0 + kPfRows, past)};
                 bool ok = mbar_wait(qfull, 0, abort_flag, p.status) && ready(0);
                 if (ok) {
                     if (n_t0 > 0) { issue_qk(0, 0); umma_commit(&sfull[0]); }
                     if (n_t1 > 0) { issue_qk(1, 0); umma_commit(&sfull[1]); }
                     umma_commit(&empty[0]);
                 }
+                // split tiles (tile 0 splits whenever tile 1 does: it sees fewer keys)
+                const int n_split = split_weights<PAGED>(p, q0 + kPfRows, past) ? 2 : split_weights<PAGED>(p, q0, past) ? 1 : 0;
                 for (int j = 0; j < nmax && ok; ++j) {
                     bool v_ready = false, k_next = false;
     #pragma unroll
@@ -333,8 +344,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                 fence_proxy_async_smem();   // generic-proxy stores before the tensor core reads
                             }
                         }
-#pragma unroll 1
-                        for (int ps = 0; ps < (split_t[t] ? 2 : 1); ++ps) issue_pv(t, 2 * j + 1, j > 0, ps > 0);
+                        issue_pv(t, 2 * j + 1, j > 0);
+                        if (t < n_split)   // the remainders: A = the upper half of S
+                            pf_issue_pv_rem(tmem + 256 + t * D, tmem + t * 128 + kPfKeys / 2,
+                                            ring_base + ((2 * j + 1) % kPfRing) * SM::kTile, SM::kHalf, idesc_pv);
                         if (j + 1 < n_t) {
                             if (!k_next) {
                                 if (!ready(2 * j + 2)) { ok = false; continue; }
@@ -393,6 +406,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const bool split = split_weights<PAGED>(p, q0 + t * kPfRows, past);   // warpgroup-uniform
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
+        // the key-tile loop, compiled twice: with the weights' bf16 remainders (a split tile)
+        // and without, so the common path carries no extra registers
+        auto tile_loop = [&](auto split_tag) {
+            constexpr bool kSplit = decltype(split_tag)::value;
         for (int j = 0; j < n_t; ++j) {
             const bool landed = mbar_wait(&sfull[t], j & 1, abort_flag, p.status);
             if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }   // tcgen05.ld/st are warp-aligned
@@ -465,19 +482,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 }
                 return w;
             };
-            if (split) {   // the remainders w - bf16(w), exact in fp32, rounded to bf16 (computed first: the main pass below
-                           // then consumes the S registers as it goes)
+            if constexpr (kSplit) {   // the remainders w - bf16(w), exact in fp32, rounded to bf16 (computed
+                                      // first: the main pass below then consumes the S registers as it goes)
 #pragma unroll
-                for (int ch = 0; ch < kPfKeys / 32; ++ch) {
-                    uint32_t rk[16];
+                for (int ch = 0; ch < kPfKeys / 16; ++ch) {
+                    uint32_t rk[8];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float2 w = weights(ch * 32 + 2 * e);
+                    for (int e = 0; e < 8; ++e) {
+                        const float2 w = weights(ch * 16 + 2 * e);
                         const float2 u = unpack_bf16x2(pack_bf16x2(w.x, w.y));
                         rk[e] = pack_bf16x2(w.x - u.x, w.y - u.y);
                         rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(rk[e]));
                     }
-                    tmem_st16(tS + kPfKeys / 2 + ch * 16, rk);
+                    tmem_st8(tS + kPfKeys / 2 + ch * 8, rk);
                 }
             }
 #pragma unroll
@@ -498,6 +515,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tc_fence_before();
             mbar_arrive(&pfull[t]);
         }
+        };
+        if (split)
+            tile_loop(std::true_type{});
+        else
+            tile_loop(std::false_type{});
         // epilogue: O / l -> bf16 -> out[b, row, head, :]
         const bool fin = n_t > 0 && ok && mbar_wait(&odone[t], 0, abort_flag, p.status);
         if (__all_sync(0xffffffffu, fin)) {

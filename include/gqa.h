@@ -37,6 +37,7 @@
 #ifndef GQA_B200_H
 #define GQA_B200_H
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -118,6 +119,48 @@ int gqa_decode(const void *q, const void *k_cache, const void *v_cache,
 int gqa_decode_rows(const void *q, const void *k_cache, const void *v_cache, int64_t cache_rows,
                     const int32_t *seqlens, void *out,
                     int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
+
+/*
+ * Decode with the batch's cached tokens divided evenly among the SMs, on the
+ * 5th-generation tensor cores: the same result as gqa_decode_rows (same
+ * arguments, same row check, same device status), built for groups of many
+ * query heads per KV head (MQA, wide GQA) and for ragged lengths.  The query
+ * heads of a group are the rows of the tensor-core products ("Multi-query
+ * attention" (pranaymahendrakar), "Why this is a bandwidth argument, not a
+ * FLOP argument": at h / n_kv query heads per KV head the step does h / n_kv
+ * multiply-adds per cached element, too many for the warp-level path once
+ * the group is wide), and a sequence whose tokens fall to several SMs is
+ * finished by the last of them, which merges the partial results
+ * (log-sum-exp rule) from the workspace.
+ *   workspace        DEVICE memory of at least
+ *                    gqa_decode_split_workspace_bytes(B, h, n_kv, d_h) bytes
+ *                    (which depends on the current device's SM count),
+ *                    256-byte aligned, owned by the caller.  Its first
+ *                    gqa_decode_split_counter_bytes(B, h, n_kv) bytes are
+ *                    arrival counters and must be zero when a call starts;
+ *                    every call leaves them zero (also after a wait timed
+ *                    out), so a workspace zero-filled once serves any number
+ *                    of calls of these sizes.  The rest is scratch.  Before a
+ *                    call whose counter bytes exceed those of the earlier
+ *                    calls, zero the extra bytes.  Calls that share a
+ *                    workspace must not overlap on the GPU (one stream, or
+ *                    ordered).
+ * Errors: as gqa_decode_rows, plus GQA_ERR_INVALID_ARG for a null,
+ * misaligned or too small workspace, GQA_ERR_UNSUPPORTED when
+ * n_kv * ceil(h / n_kv / 128) * B exceeds 2^24.
+ */
+int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache, int64_t cache_rows,
+                     const int32_t *seqlens, void *out,
+                     int B, int h, int n_kv, int d_h, float scale,
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes gqa_decode_split needs for these sizes on the current
+ * device; 0 for sizes gqa_decode_split rejects. */
+size_t gqa_decode_split_workspace_bytes(int B, int h, int n_kv, int d_h);
+
+/* Bytes at the start of the workspace that hold the arrival counters (a
+ * multiple of 256); 0 for sizes gqa_decode_split rejects. */
+size_t gqa_decode_split_counter_bytes(int B, int h, int n_kv);
 
 /*
  * Decode over an 8-bit cache ("Multi-Query Attention (MQA)" (inferensys

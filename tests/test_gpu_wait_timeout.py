@@ -76,7 +76,11 @@ def test_decode_wait_runs_out(W, B, h, n_kv, d, lens):
     launch = lambda lib: lib.gqa_decode_rows(q.data_ptr(), k.data_ptr(), v.data_ptr(), k.shape[0], L.data_ptr(),  # noqa
                                              out.data_ptr(), B, h, n_kv, d, d ** -0.5, stream())
     got = stalled_then_clean(W, launch, out)
-    assert torch.equal(got, gqa.decode(q, k, v, L))
+    want = torch.empty_like(q)    # the product library's same entry point
+    assert gqa.gqa_decode_rows(q.data_ptr(), k.data_ptr(), v.data_ptr(), k.shape[0], L.data_ptr(), want.data_ptr(),
+                               B, h, n_kv, d, d ** -0.5, stream()) == _lib.GQA_OK
+    torch.cuda.synchronize()
+    assert torch.equal(got, want)
 
 
 @pytest.mark.parametrize("fp8", [False, True], ids=["bf16", "e4m3"])
@@ -144,3 +148,20 @@ def test_mla_wait_runs_out(W):
 
 def test_product_library_status_clean():
     assert gqa.gqa_get_device_status() == _lib.GQA_OK
+
+
+def test_split_decode_wait_runs_out(W):
+    """The split-KV kernel: the stalled call times out, its workspace counters still
+    return to zero (the next call through the same workspace is exact)."""
+    B, h, n_kv, d = 6, 64, 1, 128
+    q, k, v, L = (t.cuda() for t in inputs.decode_inputs(27, B, h, n_kv, d, [3000, 10, 700, 5000, 64, 1]))
+    out = torch.empty_like(q)
+    nbytes = W.gqa_decode_split_workspace_bytes(B, h, n_kv, d)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    launch = lambda lib: lib.gqa_decode_split(q.data_ptr(), k.data_ptr(), v.data_ptr(), k.shape[0],  # noqa: E731
+                                              L.data_ptr(), out.data_ptr(), B, h, n_kv, d, d ** -0.5,
+                                              ws.data_ptr(), nbytes, stream())
+    got = stalled_then_clean(W, launch, out)
+    assert torch.equal(got, gqa.decode_split(q, k, v, L))
+    counters = ws[:W.gqa_decode_split_counter_bytes(B, h, n_kv)].view(torch.int32)   # at the workspace's start
+    assert torch.all(counters == 0)
