@@ -192,8 +192,10 @@ def prefill(q, k, v, causal: bool = True, scale: float | None = None, out=None, 
 
 # Groups of at least this many query heads per KV head, over caches holding at
 # least SPLIT_MIN_MEAN_ROWS rows per sequence, go to the split-KV tensor-core
-# kernel (gqa_decode_split); everything else to the cluster kernel.
-SPLIT_MIN_GROUP = 32
+# kernel (gqa_decode_split); everything else to the cluster kernel.  (Measured
+# on B200: the split kernel's heads-as-rows layout leaves one softmax warp per
+# 32 heads, so below 128 heads per group the cluster kernel is faster.)
+SPLIT_MIN_GROUP = 128
 SPLIT_MIN_MEAN_ROWS = 256
 _workspaces = {}   # device index -> [workspace tensor, bytes at its start known to be zero after the last call]
 

@@ -116,9 +116,10 @@ def test_split_lengths_past_the_cache_rows_are_cut_and_reported():
 
 
 def test_decode_dispatches_wide_groups_to_the_split_kernel():
-    """decode() sends groups of >= 32 heads over caches of >= 256 rows per sequence to
-    gqa_decode_split: the result is bit-identical to calling it directly."""
-    q, k, v, lens = (t.cuda() for t in inputs.decode_inputs(38, 8, 32, 1, 128, 2000))
+    """decode() sends groups of >= SPLIT_MIN_GROUP heads over caches of >= 256 rows per
+    sequence to gqa_decode_split: the result is bit-identical to calling it directly."""
+    G = _lib.SPLIT_MIN_GROUP
+    q, k, v, lens = (t.cuda() for t in inputs.decode_inputs(38, 4, G, 1, 128, 2000))
     assert torch.equal(gqa.decode(q, k, v, lens), gqa.decode_split(q, k, v, lens))
 
 
