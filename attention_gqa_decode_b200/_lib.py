@@ -22,6 +22,7 @@ SIGNATURES = {
     "gqa_decode_split": ([_vp, _vp, _vp, _i64, _vp, _vp, _i, _i, _i, _i, _f, _vp, ctypes.c_size_t, _vp], _i),
     "gqa_decode_split_workspace_bytes": ([_i, _i, _i, _i], ctypes.c_size_t),
     "gqa_decode_split_counter_bytes": ([_i, _i, _i], ctypes.c_size_t),
+    "gqa_decode_split_noalloc": ([_vp, _vp, _vp, _i64, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_fp8_rows": ([_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_paged": ([_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),

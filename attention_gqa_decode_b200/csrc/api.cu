@@ -37,6 +37,9 @@ int launch_decode_split(const void *q, const void *k, const void *v, long long c
                         cudaStream_t stream);
 size_t split_workspace_bytes(int B, int h, int n_kv, int d);
 size_t split_counter_bytes(int B, int h, int n_kv);
+int launch_decode_split_noalloc(const void *q, const void *k, const void *v, long long cache_rows,
+                                const int32_t *seqlens, void *out, int B, int h, int n_kv, int d, float scale,
+                                cudaStream_t stream);
 }  // namespace gqa
 
 namespace gqa_host {
@@ -195,6 +198,23 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache, in
     if (workspace_bytes < gqa::split_workspace_bytes(B, h, n_kv, d_h)) return GQA_ERR_INVALID_ARG;
     return gqa::launch_decode_split(q, k_cache, v_cache, cache_rows, seqlens, out, B, h, n_kv, d_h, scale, workspace,
                                     workspace_bytes, stream);
+}
+
+int gqa_decode_split_noalloc(const void *q, const void *k_cache, const void *v_cache, int64_t cache_rows,
+                             const int32_t *seqlens, void *out, int B, int h, int n_kv, int d_h, float scale,
+                             cudaStream_t stream) {
+    if (!rows_ok(cache_rows)) return GQA_ERR_INVALID_ARG;
+    if (!q || !k_cache || !v_cache || !seqlens || !out) return GQA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+        return GQA_ERR_INVALID_ARG;
+    if (B <= 0 || B > 65535 || h <= 0 || n_kv <= 0 || h % n_kv != 0) return GQA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return GQA_ERR_INVALID_ARG;
+    if (d_h != 64 && d_h != 128) return GQA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(n_kv) * ((h / n_kv + 127) / 128) * B > (1LL << 24)) return GQA_ERR_UNSUPPORTED;
+    const int st = gqa::launch_decode_split_noalloc(q, k_cache, v_cache, cache_rows, seqlens, out, B, h, n_kv, d_h,
+                                                    scale, stream);
+    return st == 0 ? GQA_OK : (st == 1 || st == 2) ? GQA_ERR_UNSUPPORTED : GQA_ERR_CUDA;
 }
 
 // Checks shared by every decode entry point (cache pointers are checked by the caller).

@@ -40,6 +40,7 @@
 // zero when a call starts; every call leaves them zero (the last arriver
 // resets its segment's counter), also when a wait times out.
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -722,6 +723,45 @@ int launch_decode_split(const void *q, const void *k, const void *v, long long c
     if (d == 128)
         return launch_split_t<128>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
     return launch_split_t<64>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
+}
+
+// ---------------------------------------------------------------------------
+// The allocation-free variant: the same kernel, with its workspace in a fixed
+// array of the library's own.  Every device that loads the library holds the
+// array (kNoAllocScratchBytes) until the process exits.
+
+constexpr size_t kNoAllocScratchBytes = 16u << 20;   // 16 MiB
+static __device__ __align__(256) unsigned char g_split_scratch[kNoAllocScratchBytes];
+
+// Device address of g_split_scratch on the current device, looked up once per
+// device (thread-safe) and kept; null if the lookup fails.
+static void *noalloc_scratch() {
+    static void *ptrs[64] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_split_scratch) != cudaSuccess) return nullptr;
+        ptrs[dev] = ptr;
+    }
+    return ptrs[dev];
+}
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// 0 = launched; 1 = the sizes need more than the fixed array; 3 = a CUDA call failed.
+int launch_decode_split_noalloc(const void *q, const void *k, const void *v, long long cache_rows,
+                                const int32_t *seqlens, void *out, int B, int h, int n_kv, int d, float scale,
+                                cudaStream_t stream) {
+    const size_t need = split_workspace_bytes(B, h, n_kv, d);
+    if (need > kNoAllocScratchBytes) return 1;
+    void *scratch = noalloc_scratch();
+    if (!scratch) return 3;
+    // the arrival counters must start at zero: clear them on the stream (the rest is scratch)
+    if (cudaMemsetAsync(scratch, 0, split_counter_bytes(B, h, n_kv), stream) != cudaSuccess) return 3;
+    return launch_decode_split(q, k, v, cache_rows, seqlens, out, B, h, n_kv, d, scale, scratch, need, stream);
 }
 
 }  // namespace gqa

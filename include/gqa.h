@@ -163,6 +163,36 @@ size_t gqa_decode_split_workspace_bytes(int B, int h, int n_kv, int d_h);
 size_t gqa_decode_split_counter_bytes(int B, int h, int n_kv);
 
 /*
+ * gqa_decode_split for callers that may not allocate device memory -- for
+ * instance a plug-in running inside another framework that must not touch
+ * that framework's memory pool, or a serving loop that forbids allocations
+ * once it has started (cudaMalloc synchronises the device and fails when the
+ * memory is fully reserved).  The paper has no counterpart: this is an
+ * interface convenience, not part of the method.
+ *   Same arguments and result as gqa_decode_split, without the workspace:
+ *   the workspace is a fixed 16 MiB array inside the library, which every
+ *   device that loads the library holds until the process exits.  The call
+ *   allocates nothing (no cudaMalloc, no allocating library routine); it
+ *   clears the array's arrival counters with cudaMemsetAsync on `stream`
+ *   before the launch.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Every call uses the same array: calls that overlap on the GPU (on
+ *   different streams, or from different threads without ordering) race and
+ *   their results are undefined.
+ * Errors: as gqa_decode_split (without the workspace checks), plus
+ * GQA_ERR_UNSUPPORTED when the sizes need more than the 16 MiB array, that is
+ * when gqa_decode_split_workspace_bytes(B, h, n_kv, d_h) exceeds 16 MiB (on a
+ * 148-SM B200: n_kv * ceil(h / n_kv / 128) * B above 104 at d_h = 128, above
+ * 348 at d_h = 64), and GQA_ERR_CUDA if the address lookup, the clear or the
+ * launch fails.  Nothing is launched on an error.
+ */
+int gqa_decode_split_noalloc(const void *q, const void *k_cache, const void *v_cache, int64_t cache_rows,
+                             const int32_t *seqlens, void *out,
+                             int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
+
+/*
  * Decode over an 8-bit cache ("Multi-Query Attention (MQA)" (inferensys
  * glossary), "KV cache quantization": the cache is kept in FP8 with scaling
  * factors; "Multi-query attention" (pranaymahendrakar), "Interaction with
