@@ -21,7 +21,6 @@ SIGNATURES = {
     "gqa_decode_rows": ([_vp, _vp, _vp, _i64, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_split": ([_vp, _vp, _vp, _i64, _vp, _vp, _i, _i, _i, _i, _f, _vp, ctypes.c_size_t, _vp], _i),
     "gqa_decode_split_workspace_bytes": ([_i, _i, _i, _i], ctypes.c_size_t),
-    "gqa_decode_split_counter_bytes": ([_i, _i, _i], ctypes.c_size_t),
     "gqa_decode_split_noalloc": ([_vp, _vp, _vp, _i64, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode_fp8_rows": ([_vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
@@ -100,10 +99,6 @@ def gqa_decode_split(q, k_cache, v_cache, cache_rows, seqlens, out, B, h, n_kv, 
 
 def gqa_decode_split_workspace_bytes(B, h, n_kv, d_h) -> int:
     return int(lib().gqa_decode_split_workspace_bytes(B, h, n_kv, d_h))
-
-
-def gqa_decode_split_counter_bytes(B, h, n_kv) -> int:
-    return int(lib().gqa_decode_split_counter_bytes(B, h, n_kv))
 
 
 def gqa_decode_fp8_rows(q, k_cache, v_cache, cache_rows, k_scale, v_scale, seqlens, out, B, h, n_kv, d_h, scale,
@@ -191,33 +186,54 @@ def prefill(q, k, v, causal: bool = True, scale: float | None = None, out=None, 
     return out
 
 
-# Groups of at least this many query heads per KV head, over caches holding at
-# least SPLIT_MIN_MEAN_ROWS rows per sequence, go to the split-KV tensor-core
-# kernel (gqa_decode_split); everything else to the cluster kernel.  (Measured
-# on B200: the split kernel's heads-as-rows layout leaves one softmax warp per
-# 32 heads, so below 128 heads per group the cluster kernel is faster.)
+# decode() sends a call to the split-KV kernels (gqa_decode_split) when the cache holds
+# at least SPLIT_MIN_MEAN_ROWS rows per sequence and either the groups are wide
+# (>= SPLIT_MIN_GROUP query heads per KV head) or there are too few (sequence, KV
+# head) units for the cluster kernel's at most 8 splits each to reach every SM;
+# everything else goes to the cluster kernel (gqa_decode_rows).  Measured on B200:
+# G = 128: split 1.6 TB/s, cluster 1.1; B4 h64 n_kv1 L32768: split 1.5 TB/s, cluster
+# 0.4; the GQA and MQA decode workloads: cluster 5.6 / 4.3, split 4.4 / 3.9.
 SPLIT_MIN_GROUP = 128
 SPLIT_MIN_MEAN_ROWS = 256
-_workspaces = {}   # device index -> [workspace tensor, bytes at its start known to be zero after the last call]
+_sm_counts = {}
 
 
-def split_workspace(device, nbytes: int, counter_bytes: int):
-    """A device workspace of at least nbytes for gqa_decode_split whose first
-    counter_bytes are zero: one per device, kept and grown as needed (every call
-    leaves its counters zero; a call with more counters than the earlier ones gets
-    the extra bytes zeroed first).  Calls that share it must not overlap on the GPU.
-    Make the first call of a shape before capturing a CUDA graph that uses it."""
+def _sm_count(device) -> int:
     import torch
     dev = torch.device(device)
     key = dev.index if dev.index is not None else torch.cuda.current_device()
-    ent = _workspaces.get(key)
-    if ent is None or ent[0].numel() < nbytes:
-        ent = [torch.zeros(max(nbytes, 1), dtype=torch.uint8, device=torch.device("cuda", key)), nbytes]
-        _workspaces[key] = ent
-    if counter_bytes > ent[1]:
-        ent[0][ent[1]:counter_bytes].zero_()
-    ent[1] = counter_bytes   # after the call only its own counters are known zero (the rest is scratch)
-    return ent[0]
+    if key not in _sm_counts:
+        _sm_counts[key] = torch.cuda.get_device_properties(key).multi_processor_count
+    return _sm_counts[key]
+
+
+def use_split(q, k_cache) -> bool:
+    """The dispatch rule of decode() for q [B, h, d] and packed caches [T, n_kv, d]."""
+    B, h, _ = q.shape
+    T, n_kv, _ = k_cache.shape
+    if n_kv <= 0 or h % n_kv or T < SPLIT_MIN_MEAN_ROWS * B:
+        return False
+    G = h // n_kv
+    units = B * n_kv * -(-G // 64)
+    return G >= SPLIT_MIN_GROUP or units * 8 < _sm_count(q.device)
+
+
+_workspaces = {}   # device index -> workspace tensor
+
+
+def split_workspace(device, nbytes: int):
+    """A device workspace of at least nbytes for gqa_decode_split: one per device, kept
+    and grown as needed (it is scratch, so it needs no initialisation).  Calls that share
+    it must not overlap on the GPU.  Make the first call of a shape before capturing a
+    CUDA graph that uses it."""
+    import torch
+    dev = torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=torch.device("cuda", key))
+        _workspaces[key] = ws
+    return ws
 
 
 def decode_split(q, k_cache, v_cache, seqlens, scale: float | None = None, out=None, stream=None, workspace=None):
@@ -242,8 +258,7 @@ def decode_split(q, k_cache, v_cache, seqlens, scale: float | None = None, out=N
             raise ValueError("out must have q's shape")
     with torch.cuda.device(q.device):
         need = gqa_decode_split_workspace_bytes(B, h, n_kv, d)
-        ws = workspace if workspace is not None else \
-            split_workspace(q.device, need, gqa_decode_split_counter_bytes(B, h, n_kv))
+        ws = workspace if workspace is not None else split_workspace(q.device, need)
         st = gqa_decode_split(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), T, seqlens.data_ptr(),
                               out.data_ptr(), B, h, n_kv, d, scale, ws.data_ptr(), ws.numel() * ws.element_size(),
                               _stream_ptr(stream))
@@ -257,14 +272,11 @@ def decode(q, k_cache, v_cache, seqlens, scale: float | None = None, out=None, s
 
     Returns out [B,h,d].  Sequence b's tokens start at cache row sum(seqlens[:b]);
     a sequence that would end past row T is cut there and GQA_ERR_INVALID_ARG is
-    recorded in the device status word (gqa_get_device_status).  Groups of
-    SPLIT_MIN_GROUP or more query heads per KV head over caches of at least
-    SPLIT_MIN_MEAN_ROWS rows per sequence run on gqa_decode_split, the rest on
-    gqa_decode_rows (the lengths stay on the device; the choice uses the shapes).
+    recorded in the device status word (gqa_get_device_status).  The call runs on
+    gqa_decode_split or gqa_decode_rows by :func:`use_split` (the lengths stay on the
+    device; the choice uses the shapes).
     """
-    if q.dim() == 3 and k_cache.dim() == 3 and k_cache.shape[1] > 0 and \
-            q.shape[1] // max(k_cache.shape[1], 1) >= SPLIT_MIN_GROUP and \
-            k_cache.shape[0] >= SPLIT_MIN_MEAN_ROWS * q.shape[0]:
+    if q.dim() == 3 and k_cache.dim() == 3 and q.is_cuda and use_split(q, k_cache):
         return decode_split(q, k_cache, v_cache, seqlens, scale=scale, out=out, stream=stream)
     import torch
     _check(q, "q", 3), _check(k_cache, "k_cache", 3), _check(v_cache, "v_cache", 3)

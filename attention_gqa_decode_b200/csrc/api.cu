@@ -36,7 +36,6 @@ int launch_decode_split(const void *q, const void *k, const void *v, long long c
                         void *out, int B, int h, int n_kv, int d, float scale, void *workspace, size_t ws_bytes,
                         cudaStream_t stream);
 size_t split_workspace_bytes(int B, int h, int n_kv, int d);
-size_t split_counter_bytes(int B, int h, int n_kv);
 int launch_decode_split_noalloc(const void *q, const void *k, const void *v, long long cache_rows,
                                 const int32_t *seqlens, void *out, int B, int h, int n_kv, int d, float scale,
                                 cudaStream_t stream);
@@ -176,11 +175,6 @@ int gqa_decode_rows(const void *q, const void *k_cache, const void *v_cache, int
 size_t gqa_decode_split_workspace_bytes(int B, int h, int n_kv, int d_h) {
     if (B <= 0 || B > 65535 || h <= 0 || n_kv <= 0 || h % n_kv != 0 || (d_h != 64 && d_h != 128)) return 0;
     return gqa::split_workspace_bytes(B, h, n_kv, d_h);
-}
-
-size_t gqa_decode_split_counter_bytes(int B, int h, int n_kv) {
-    if (B <= 0 || B > 65535 || h <= 0 || n_kv <= 0 || h % n_kv != 0) return 0;
-    return gqa::split_counter_bytes(B, h, n_kv);
 }
 
 int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache, int64_t cache_rows,

@@ -25,20 +25,21 @@
 //     the sequence boundaries.  A CTA's range is a run of segments (pieces of
 //     sequences); a segment wholly inside one CTA is finished there, the
 //     pieces of a segment cut between CTAs leave partial results (running
-//     max, running sum, unnormalised O) in the caller's workspace, and the
-//     last CTA to finish a piece of that segment (an arrival counter per
-//     segment) merges them with the log-sum-exp rule and writes the output;
+//     max, running sum, unnormalised O) in the caller's workspace, and a
+//     second, small kernel merges them with the log-sum-exp rule, one block
+//     per (segment, head) on every SM at once;
 //   - roles: warp 4 streams Q (once per segment) and K/V stages with TMA into
 //     a ring, warp 5 allocates TMEM and issues the MMAs, warps 0-3 run the
 //     softmax (lazy rescale: the running max moves only when a row's stage
 //     max exceeds it by 2^8) and the epilogue.  S is double-buffered in TMEM,
 //     so Q K^T of stage i + 1 runs while the softmax of stage i does.
-// Workspace: one arrival counter per segment first (padded to 256 bytes),
-// then the partial slots (CTA c's piece of segment s goes to slot c + s --
-// each CTA's segments and each segment's CTAs are runs, so the (CTA,
-// segment) pairs form a staircase and c + s is unique).  The counters must be
-// zero when a call starts; every call leaves them zero (the last arriver
-// resets its segment's counter), also when a wait times out.
+// Workspace: one record per segment first (the CTAs of its first and last
+// piece, written by the CTA of the first piece; (-1, -1) for an empty
+// sequence), padded to 256 bytes, then the partial slots (CTA c's piece of
+// segment s goes to slot c + s -- each CTA's segments and each segment's CTAs
+// are runs, so the (CTA, segment) pairs form a staircase and c + s is
+// unique).  Every call writes what it reads: the workspace needs no
+// initialisation.
 #include <algorithm>
 #include <mutex>
 
@@ -73,7 +74,7 @@ struct SplitParams {
     const int32_t *seqlens;      // [B]
     __nv_bfloat16 *out;          // [B, h, D]
     float *part;                 // workspace: partial slots
-    int *count;                  // workspace: one arrival counter per segment
+    int2 *seg;                   // workspace: per segment, the CTAs of its first and last piece
     int B, h, n_kv, G, slices, nctas;
     uint32_t q_bytes;            // bytes of one Q box (min(128, h) heads)
     long long cache_rows;
@@ -168,7 +169,6 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     long long *scan = reinterpret_cast<long long *>(drain + 2);   // [8]: block-scan scratch (after tmem/abort)
-    int *flag = reinterpret_cast<int *>(scan + 8);                // [1]: last-arriver broadcast
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x, NC = p.nctas;
@@ -225,6 +225,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
             if (bb < p.B && cut == 0 && bb % NC == c) {   // no tokens: a zero output row for every head
                 uint4 *o4 = reinterpret_cast<uint4 *>(p.out + static_cast<size_t>(bb) * p.h * D);
                 for (int i = 0; i < p.h * D / 8; ++i) o4[i] = make_uint4(0u, 0u, 0u, 0u);
+                for (int gs = 0; gs < p.n_kv * p.slices; ++gs) p.seg[gs * p.B + bb] = make_int2(-1, -1);
             }
             // block-wide sum of the cut lengths
             long long s = cut;
@@ -577,48 +578,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(ofree);
             ++seg;
-            if (!whole) {
-                // arrival: the last of the segment's pieces merges them (also after a timeout,
-                // so that every counter returns to zero; the outputs are then unspecified)
-                __threadfence();
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (threadIdx.x == 0) {
-                    const int prev = atomicAdd(&p.count[sidx], 1);
-                    const int last = prev == last_c - first_c;
-                    if (last) p.count[sidx] = 0;
-                    *flag = last;
-                }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (*reinterpret_cast<volatile int *>(flag)) {
-                    __threadfence();
-                    if (r < HS) {
-                        float M = -INFINITY;
-                        for (int cc = first_c; cc <= last_c; ++cc)
-                            M = fmaxf(M, __ldcg(p.part + static_cast<size_t>(cc + sidx) * SG::kPartFloats + kSpRows * D + r));
-                        float Lsum = 0.f;
-                        for (int cc = first_c; cc <= last_c; ++cc) {
-                            const float *sp = p.part + static_cast<size_t>(cc + sidx) * SG::kPartFloats;
-                            Lsum += exp2f(__ldcg(sp + kSpRows * D + r) - M) * __ldcg(sp + kSpRows * D + kSpRows + r);
-                        }
-                        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-                        __nv_bfloat16 *orow = p.out + (static_cast<size_t>(sg.b) * p.h + head0 + r) * D;
-                        for (int ch = 0; ch < D / 8; ++ch) {
-                            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                            for (int cc = first_c; cc <= last_c; ++cc) {
-                                const float *sp = p.part + static_cast<size_t>(cc + sidx) * SG::kPartFloats;
-                                const float wgt = exp2f(__ldcg(sp + kSpRows * D + r) - M);
-                                const float4 a = __ldcg(reinterpret_cast<const float4 *>(sp + static_cast<size_t>(r) * D + ch * 8));
-                                const float4 b = __ldcg(reinterpret_cast<const float4 *>(sp + static_cast<size_t>(r) * D + ch * 8 + 4));
-                                acc[0] += wgt * a.x; acc[1] += wgt * a.y; acc[2] += wgt * a.z; acc[3] += wgt * a.w;
-                                acc[4] += wgt * b.x; acc[5] += wgt * b.y; acc[6] += wgt * b.z; acc[7] += wgt * b.w;
-                            }
-                            *reinterpret_cast<uint4 *>(orow + ch * 8) =
-                                make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                                           pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
-                        }
-                    }
-                }
-            }
+            // the segment's record for the merge kernel, from the CTA of its first piece
+            if (c == first_c && threadIdx.x == 0) p.seg[sidx] = make_int2(first_c, last_c);
         }
     }
 
@@ -631,24 +592,643 @@ __global__ void __launch_bounds__(kSpThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Tokens as rows, for groups of at most 64 heads (d = 128).  With the heads
+// as the rows, a group of 32 heads leaves its softmax to one warp of the
+// four that can reach its TMEM lanes; here a stage's 128 tokens are the M
+// rows instead, so all four softmax warps share the work:
+//   S^T = K Q^T        M = 128 tokens, N = 64 heads (padded), K = d      (TMEM)
+//   P^T = exp2(S^T c - m)  per column (head), thread = token row, written as
+//                      bf16 to shared memory (token rows of 64 heads)
+//   O^T += V^T P^T     M = 128 (d), N = 64 heads, K = 128 tokens; A = V read
+//                      MN-major from the stage's tile, B = P^T        (TMEM)
+// The running max per head is lazy: taken over the segment's first stage
+// (a column max across the 128 token threads), it moves only when a score
+// passes it by more than 2^8 (a vote among the softmax warps; then the O^T
+// columns and the sums are rescaled).  Each thread keeps its own partial
+// column sums; they are reduced across the threads when the segment ends.
+// K and V stream through one ring of 32 KB items (K(i) = item 2i, V(i) =
+// item 2i + 1), so a K tile is released as soon as its Q K^T is done.
+
+constexpr int kTkTok = 128;              // tokens per stage: MMA M of S^T = K Q^T
+constexpr int kTkN = 64;                 // MMA N: the slice's heads, padded
+constexpr int kTkItems = 6;              // ring of K / V items
+constexpr uint32_t kTkTmemCols = 256;    // S^T [0, 64) and [64, 128); O^T [128, 192)
+constexpr float kTkRescale = 8.0f;       // lazy rescale threshold (log2 units)
+
+struct TokGeom {                         // D = 128
+    static constexpr int D = 128;
+    static constexpr uint32_t kQPanel = kTkN * 128;        // Q: 2 panels of 64 heads x 128 B
+    static constexpr uint32_t kQ = 2 * kQPanel;
+    static constexpr uint32_t kItemPanel = kTkTok * 128;   // K or V of a stage: 2 panels of 128 tokens x 128 B
+    static constexpr uint32_t kItem = 2 * kItemPanel;
+    static constexpr uint32_t kP = kTkTok * 128;           // P^T: 128 token rows of 64 bf16 heads, 128B swizzled
+    static constexpr uint32_t kRed = 4 * kTkN * 4;         // [4 warps][64 heads] float exchange buffer
+    static constexpr uint32_t kMsh = kTkN * 4;             // running max per head
+    static constexpr uint32_t kCres = kTkN * 4;            // a column reduction's 64 results
+    static constexpr uint32_t kCtrl = 512;
+    static constexpr uint32_t kTotal = kQ + kP + kTkItems * kItem + kRed + kMsh + kCres + kCtrl + 1024;
+    static constexpr uint32_t kPartFloats = SplitGeom<128>::kPartFloats;   // the workspace slot of the other kernel
+};
+static_assert(TokGeom::kTotal <= 232448, "shared memory of the tokens-as-rows kernel");
+
+template <int NH>   // the slice's heads as the N of S^T = K Q^T: 16, 32 or 64 (the group, rounded up)
+__global__ void __launch_bounds__(kSpThreads, 1)
+    gqa_decode_split_tok_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                                const __grid_constant__ CUtensorMap tm_v, const SplitParams p) {
+    using TG = TokGeom;
+    constexpr int D = TG::D;
+    constexpr int R = kTkItems;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem;
+    uint8_t *sP = sQ + TG::kQ;
+    uint8_t *sRing = sP + TG::kP;
+    float *red = reinterpret_cast<float *>(sRing + R * TG::kItem);   // [4][64]
+    float *msh = red + 4 * kTkN;                                  // [64] running max (log2 units)
+    float *cres = msh + kTkN;                                     // [64] a column reduction's results
+    uint64_t *bars = reinterpret_cast<uint64_t *>(cres + kTkN);
+    uint64_t *qfull = bars;
+    uint64_t *qfree = qfull + 1;
+    uint64_t *full = qfree + 1;            // [R]
+    uint64_t *empty = full + R;            // [R]
+    uint64_t *sfull = empty + R;           // [2] S^T buffer written
+    uint64_t *sfree = sfull + 2;           // [2] S^T buffer read by every softmax warp
+    uint64_t *pfull = sfree + 2;           // P^T published (one arrival per softmax warp per publication)
+    uint64_t *pvdone = pfull + 1;          // every P V, in order (phase k = publication k)
+    uint64_t *ofree = pvdone + 1;          // the segment's O^T read out (one arrival per warp)
+    uint64_t *drain = ofree + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    long long *scan = reinterpret_cast<long long *>(drain + 2);   // [8]
+    int *vote = reinterpret_cast<int *>(scan + 8);                // [3] rescale votes, by stage % 3
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x, NC = p.nctas;
+
+    if (threadIdx.x == 0) {
+        mbar_init(qfull, 1);
+        mbar_init(qfree, 1);
+        for (int i = 0; i < R; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sfull[i], 1);
+            mbar_init(&sfree[i], 4);
+        }
+        mbar_init(pfull, 4);
+        mbar_init(pvdone, 1);
+        mbar_init(ofree, 4);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        vote[0] = vote[1] = vote[2] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, kTkTmemCols);
+        tmem_relinquish();
+    }
+    // P^T columns NH..63 are read by P V (N = 64) and never written: zero them once
+    for (int i = threadIdx.x; i < static_cast<int>(TG::kP / 16); i += kSpThreads)
+        reinterpret_cast<uint4 *>(sP)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+
+    // ---- T = sum of the cut lengths; zero rows for sequences with no tokens (as the other kernel)
+    long long T = 0;
+    {
+        long long base_off = 0;
+        for (int b0 = 0; b0 < p.B; b0 += kSpThreads) {
+            const int bb = b0 + threadIdx.x;
+            const long long l = bb < p.B ? max(p.seqlens[bb], 0) : 0;
+            long long x = l;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (lane == 31) scan[warp] = x;
+            __syncthreads();
+            long long before = 0, chunk = 0;
+            for (int w = 0; w < kSpThreads / 32; ++w) {
+                if (w < warp) before += scan[w];
+                chunk += scan[w];
+            }
+            const long long off_b = base_off + before + x - l;
+            const long long cut = bb < p.B ? max(0LL, min(l, p.cache_rows - off_b)) : 0;
+            if (cut < l) record_status(p.status, kStatusInvalid);
+            if (bb < p.B && cut == 0 && bb % NC == c) {
+                uint4 *o4 = reinterpret_cast<uint4 *>(p.out + static_cast<size_t>(bb) * p.h * D);
+                for (int i = 0; i < p.h * D / 8; ++i) o4[i] = make_uint4(0u, 0u, 0u, 0u);
+                for (int gs = 0; gs < p.n_kv * p.slices; ++gs) p.seg[gs * p.B + bb] = make_int2(-1, -1);
+            }
+            long long s = cut;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            __syncthreads();
+            if (lane == 0) scan[warp] = s;
+            __syncthreads();
+            for (int w = 0; w < kSpThreads / 32; ++w) T += scan[w];
+            base_off += chunk;
+            __syncthreads();
+        }
+    }
+    const long long W = static_cast<long long>(p.n_kv) * p.slices * T;
+    const int NCe = W < NC ? static_cast<int>(W) : NC;
+    const long long w_lo = c < NCe ? W * c / NCe : W, w_hi = c < NCe ? W * (c + 1) / NCe : W;
+    const float cl2 = p.scale_log2;
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    auto cursor = [&]() {
+        SplitCursor cu;
+        cu.p = &p;
+        cu.T = T;
+        cu.w_cur = w_lo;
+        cu.w_hi = w_hi;
+        cu.gs = 0;
+        cu.b = 0;
+        cu.off = 0;
+        cu.wb = 0;
+        if (T > 0) {
+            cu.gs = static_cast<int>(w_lo / T);
+            long long r = w_lo - cu.gs * T;
+            while (cu.b < p.B) {
+                const int L = cu.cut_len(cu.b, cu.off);
+                if (r < L) break;
+                r -= L;
+                cu.wb += L;
+                cu.off += max(p.seqlens[cu.b], 0);
+                ++cu.b;
+            }
+        }
+        return cu;
+    };
+    auto n_stages = [](const SplitSeg &sg) { return (sg.t1 - sg.t0 + kTkTok - 1) / kTkTok; };
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            SplitCursor cu = cursor();
+            SplitSeg sg;
+            int it = 0, seg = 0;
+            const int first_loaded = GQA_STALLED(p) ? 1 : 0;   // wait-test build: item 0 never arrives
+            bool ok = true;
+            while (ok && cu.next(sg)) {
+                const int g = sg.gs / p.slices;
+                const int head0 = g * p.G;
+                if (seg > 0 && !mbar_wait(qfree, (seg - 1) & 1, abort_flag, p.status)) break;
+                mbar_arrive_expect_tx(qfull, p.q_bytes);
+                for (int hf = 0; hf < D / 64; ++hf)
+                    tma_load_3d(sQ + hf * TG::kQPanel, &tm_q, qfull, hf * 64, head0, sg.b);
+                ++seg;
+                const int n = n_stages(sg);
+                for (int i = 0; i < n && ok; ++i) {
+                    const int z = static_cast<int>(sg.off) + sg.t0 + i * kTkTok;   // first cache row of the stage
+                    for (int kv = 0; kv < 2; ++kv, ++it) {
+                        const int slot = it % R, use = it / R;
+                        if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, abort_flag, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        if (it < first_loaded) continue;
+                        uint8_t *dst = sRing + slot * TG::kItem;
+                        mbar_arrive_expect_tx(&full[slot], TG::kItem);
+                        for (int hf = 0; hf < D / 64; ++hf)
+                            tma_load_3d(dst + hf * TG::kItemPanel, kv ? &tm_v : &tm_k, &full[slot], hf * 64, g, z);
+                    }
+                }
+            }
+            if (*abort_flag) {   // let the copies in flight land before the CTA moves on
+                if (seg > 0) mbar_wait_drain(qfull, (seg - 1) & 1, p.status);
+                for (int i = max(first_loaded, it - R); i < it; ++i)
+                    mbar_wait_drain(&full[i % R], (i / R) & 1, p.status);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer (warp-wide, lane 0 issues)
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(kTkTok, NH, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(kTkTok, kTkN, true, true);
+        const uint32_t q_base = smem_u32(sQ);
+        const uint32_t p_base = smem_u32(sP);
+        const uint32_t ring_base = smem_u32(sRing);
+        auto wait1 = [&](uint64_t *bar, uint32_t parity) -> bool {
+            int r = 1;
+            if (lane == 0) r = mbar_wait(bar, parity, abort_flag, p.status);
+            return __shfl_sync(0xffffffffu, r, 0) != 0;
+        };
+        auto issue_qk = [&](int gi) {   // S^T[gi % 2] = K(gi) Q^T
+            const uint32_t a0 = ring_base + ((2 * gi) % R) * TG::kItem;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+                umma_ss(tmem + (gi & 1) * kTkN,
+                        sdesc_sw128(a0 + (ks >> 2) * TG::kItemPanel + (ks & 3) * 32, 16, 1024),
+                        sdesc_sw128(q_base + (ks >> 2) * TG::kQPanel + (ks & 3) * 32, 16, 1024), idesc_qk, ks > 0);
+        };
+        auto issue_pv = [&](int gi, bool acc) {   // O^T (+)= V(gi)^T P^T
+            const uint32_t a0 = ring_base + ((2 * gi + 1) % R) * TG::kItem;
+#pragma unroll
+            for (int kk = 0; kk < kTkTok / 16; ++kk)
+                umma_ss(tmem + 2 * kTkN, sdesc_sw128(a0 + kk * 16 * 128, TG::kItemPanel, 1024),
+                        sdesc_sw128(p_base + kk * 16 * 128, TG::kItemPanel, 1024), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        };
+        SplitCursor cu = cursor();
+        SplitSeg sg;
+        int gi0 = 0, seg = 0, pub = 0;
+        bool ok = true;
+        while (ok && cu.next(sg)) {
+            const int n = n_stages(sg);
+            const int pubs = sg.L <= kSpSplitAllBelow ? 2 : 1;   // P^T published once, or twice (bf16 + remainders)
+            ok = wait1(qfull, seg & 1);
+            for (int i = 0; i < min(n, 2) && ok; ++i) {
+                ok = wait1(&full[(2 * (gi0 + i)) % R], ((2 * (gi0 + i)) / R) & 1);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    issue_qk(gi0 + i);
+                    umma_commit(&sfull[(gi0 + i) & 1]);
+                    umma_commit(&empty[(2 * (gi0 + i)) % R]);
+                    if (i == n - 1) umma_commit(qfree);
+                }
+                __syncwarp();
+            }
+            for (int i = 0; i < n && ok; ++i) {
+                const int gi = gi0 + i;
+                if (i + 2 < n) {   // Q K^T two stages ahead, as soon as S^T(gi) has been read
+                    ok = wait1(&sfree[gi & 1], (gi >> 1) & 1) && wait1(&full[(2 * (gi + 2)) % R], ((2 * (gi + 2)) / R) & 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        issue_qk(gi + 2);
+                        umma_commit(&sfull[gi & 1]);
+                        umma_commit(&empty[(2 * (gi + 2)) % R]);
+                        if (i + 2 == n - 1) umma_commit(qfree);
+                    }
+                    __syncwarp();
+                }
+                ok = wait1(&full[(2 * gi + 1) % R], ((2 * gi + 1) / R) & 1);
+                if (ok && i == 0 && seg > 0) ok = wait1(ofree, (seg - 1) & 1);   // the last segment's O^T is read out
+                if (!ok) break;
+                const int valid = min(kTkTok, sg.t1 - (sg.t0 + i * kTkTok));
+                if (valid < kTkTok) {   // V rows past the segment's tokens: cleared (0 * whatever adds nothing)
+                    uint8_t *vt = sRing + ((2 * gi + 1) % R) * TG::kItem;
+                    for (int hf = 0; hf < D / 64; ++hf)
+                        for (int e = lane; e < (kTkTok - valid) * 8; e += 32) {
+                            const int r = valid + e / 8, ch = e % 8;
+                            *reinterpret_cast<uint4 *>(vt + hf * TG::kItemPanel + r * 128 + ch * 16) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                for (int ps = 0; ps < pubs && ok; ++ps, ++pub) {
+                    ok = wait1(pfull, pub & 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        issue_pv(gi, i > 0 || ps > 0);
+                        if (ps == pubs - 1) umma_commit(&empty[(2 * gi + 1) % R]);
+                        umma_commit(pvdone);
+                    }
+                    __syncwarp();
+                }
+            }
+            gi0 += n;
+            ++seg;
+        }
+        if (!ok && lane == 0) {
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0, p.status);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue (warps 0-3)
+        const int r = warp * 32 + lane;                                  // TMEM lane: token row of S^T, d of O^T
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t tO = tmem + 2 * kTkN + lane_off;
+        const int tid = threadIdx.x;                                      // 0..127
+        SplitCursor cu = cursor();
+        SplitSeg sg;
+        int gi0 = 0, pub = 0;
+        bool ok = true;
+        // NH consecutive 32-bit TMEM columns of this thread's lane
+        auto tmem_row = [&](uint32_t taddr, float (&x)[NH]) {
+            if constexpr (NH == 16) {
+                uint32_t raw[16];
+                tmem_ld16(taddr, raw);
+                tmem_wait_ld();
+#pragma unroll
+                for (int h = 0; h < 16; ++h) x[h] = __uint_as_float(raw[h]);
+            } else {
+#pragma unroll
+                for (int q32 = 0; q32 < NH / 32; ++q32) {
+                    uint32_t raw[32];
+                    tmem_ld32(taddr + q32 * 32, raw);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < 32; ++h) x[q32 * 32 + h] = __uint_as_float(raw[h]);
+                }
+            }
+        };
+        // column reduction over the 128 token threads of NH per-thread values (max or sum)
+        // into dst[NH] in shared memory (each use separated from the next by a barrier)
+        auto colreduce = [&](const float (&x)[NH], bool is_max, float *dst) {
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                float v = x[h];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const float u = __shfl_xor_sync(0xffffffffu, v, o);
+                    v = is_max ? fmaxf(v, u) : v + u;
+                }
+                if (lane == 0) red[warp * kTkN + h] = v;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (tid < NH) {
+                const float a = red[tid], b2 = red[kTkN + tid], c2 = red[2 * kTkN + tid], d2 = red[3 * kTkN + tid];
+                dst[tid] = is_max ? fmaxf(fmaxf(a, b2), fmaxf(c2, d2)) : (a + b2) + (c2 + d2);
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+        };
+        auto load_m = [&](float (&m)[NH]) {
+#pragma unroll
+            for (int h = 0; h < NH; h += 4) {
+                const float4 v4 = *reinterpret_cast<const float4 *>(msh + h);
+                m[h] = v4.x;
+                m[h + 1] = v4.y;
+                m[h + 2] = v4.z;
+                m[h + 3] = v4.w;
+            }
+        };
+        while (cu.next(sg)) {
+            const int g = sg.gs / p.slices;
+            const int head0 = g * p.G;
+            const int HS = min(p.G, NH);
+            const int n = n_stages(sg);
+            const bool split = sg.L <= kSpSplitAllBelow;
+            float2 ls[NH / 2];   // this thread's share of the column sums
+#pragma unroll
+            for (int j = 0; j < NH / 2; ++j) ls[j] = make_float2(0.f, 0.f);
+            // the running max per head (log2 units): msh, copied into registers when they allow
+            constexpr bool kMReg = NH <= 32;
+            float m[kMReg ? NH : 1];
+            auto mv = [&](int h) -> float {
+                if constexpr (kMReg) return m[h];
+                else return msh[h];
+            };
+            for (int i = 0; i < n && ok; ++i) {
+                const int gi = gi0 + i;
+                const bool landed = mbar_wait(&sfull[gi & 1], (gi >> 1) & 1, abort_flag, p.status);
+                if (!__all_sync(0xffffffffu, landed)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                float x[NH];
+                tmem_row(tmem + (gi & 1) * kTkN + lane_off, x);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfree[gi & 1]);   // S^T(gi) may be overwritten
+                const int valid = min(kTkTok, sg.t1 - (sg.t0 + i * kTkTok));
+                const bool tok_ok = r < valid;
+                if (i == 0) {   // the segment's running max starts at its first stage's column max
+                    float xs[NH];
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) xs[h] = tok_ok ? x[h] * cl2 : -INFINITY;
+                    colreduce(xs, true, msh);
+                    if constexpr (kMReg) load_m(m);
+                }
+                // exponent arguments e = S c - m, in place, and this thread's largest (real heads)
+                float emax = -INFINITY;
+#pragma unroll
+                for (int h = 0; h < NH; h += 2) {
+                    const float2 e = ffma2(x[h], x[h + 1], cl2, -mv(h), -mv(h + 1));
+                    x[h] = e.x;
+                    x[h + 1] = e.y;
+                    emax = fmax3(emax, h < HS ? e.x : -INFINITY, h + 1 < HS ? e.y : -INFINITY);
+                }
+                // vote[gi % 3] collects this stage's votes; after the barrier everyone reads it,
+                // and vote[(gi + 2) % 3] -- read at the stage before this one, written next at
+                // the stage after the next barrier -- is cleared
+                bool rescale = false;
+                if (i > 0) {
+                    if (__any_sync(0xffffffffu, tok_ok && emax > kTkRescale) && lane == 0) atomicOr(&vote[gi % 3], 1);
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    rescale = *reinterpret_cast<volatile int *>(&vote[gi % 3]) != 0;
+                }
+                if (tid == 0) vote[(gi + 2) % 3] = 0;
+                if (rescale) {
+                    // the new column max (into cres); O^T (after the last P V), the sums and the
+                    // exponent arguments move to it
+                    {
+                        float xs[NH];
+#pragma unroll
+                        for (int h = 0; h < NH; ++h) xs[h] = tok_ok ? x[h] + mv(h) : -INFINITY;
+                        colreduce(xs, true, cres);
+                    }
+                    const bool pv_ok = mbar_wait(pvdone, (pub - 1) & 1, abort_flag, p.status);
+                    if (!__all_sync(0xffffffffu, pv_ok)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        const float mo = mv(h), mn = fmaxf(mo, cres[h]);
+                        const float a = exp2f(mo - mn);
+                        x[h] += mo - mn;
+                        if (h & 1) ls[h / 2].y *= a; else ls[h / 2].x *= a;
+                        if constexpr (kMReg) m[h] = mn;   // (msh keeps the old max until below)
+                    }
+#pragma unroll 1
+                    for (int q8 = 0; q8 < NH / 8; ++q8) {   // O^T columns in groups of 8
+                        uint32_t raw[8];
+                        tmem_ld8(tO + q8 * 8, raw);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int h = q8 * 8 + e;
+                            const float mo = msh[h], mn = fmaxf(mo, cres[h]);
+                            raw[e] = __float_as_uint(__uint_as_float(raw[e]) * exp2f(mo - mn));
+                        }
+                        tmem_st8(tO + q8 * 8, raw);
+                    }
+                    tmem_wait_st();
+                    asm volatile("bar.sync 1, 128;" ::: "memory");   // every thread has read msh and cres
+                    if (tid < NH) msh[tid] = fmaxf(msh[tid], cres[tid]);
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                }
+                // P^T row of this token: the weights exp2(e) of the HS heads (0 past them and for
+                // rows past the segment's tokens); twice for a split segment (bf16, then the bf16
+                // remainders), each after the previous P V has read the buffer
+                for (int ps = 0; ps < (split ? 2 : 1); ++ps, ++pub) {
+                    if (pub > 0) {   // the previous P V has read the buffer
+                        const bool pv_ok = mbar_wait(pvdone, (pub - 1) & 1, abort_flag, p.status);
+                        if (!__all_sync(0xffffffffu, pv_ok)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    uint8_t *prow = sP + r * 128;
+#pragma unroll
+                    for (int ch = 0; ch < NH / 8; ++ch) {   // 8 heads per 16-byte chunk of the row
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int h = ch * 8 + 2 * e2;
+                            float w0 = tok_ok && h < HS ? exp2f(x[h]) : 0.f;
+                            float w1 = tok_ok && h + 1 < HS ? exp2f(x[h + 1]) : 0.f;
+                            uint32_t q2 = pack_bf16x2(w0, w1);
+                            if (ps == 1) {   // the remainders w - bf16(w), exact in fp32
+                                const float2 u = unpack_bf16x2(q2);
+                                q2 = pack_bf16x2(w0 - u.x, w1 - u.y);
+                            }
+                            ls[h / 2] = fadd2(ls[h / 2], unpack_bf16x2(q2));
+                            pk[e2] = q2;
+                        }
+                        *reinterpret_cast<uint4 *>(prow + (((ch ^ r) & 7) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(pfull);
+                }
+            }
+            gi0 += n;
+
+            // ---- epilogue: column sums, O^T, then the output or a partial result
+            const int first_c = split_owner(sg.w, W, NCe), last_c = split_owner(sg.w + sg.L - 1, W, NCe);
+            const bool whole = first_c == last_c;
+            const int sidx = sg.gs * p.B + sg.b;
+            float *slot = p.part + static_cast<size_t>(c + sidx) * TG::kPartFloats;
+            {
+                float lf[NH];
+#pragma unroll
+                for (int j = 0; j < NH / 2; ++j) {
+                    lf[2 * j] = ls[j].x;
+                    lf[2 * j + 1] = ls[j].y;
+                }
+                colreduce(lf, false, cres);   // cres[h] = the segment's column sum of head h
+            }
+            bool have_o = false;
+            if (ok) {
+                const bool fin = mbar_wait(pvdone, (pub - 1) & 1, abort_flag, p.status);
+                have_o = __all_sync(0xffffffffu, fin);
+                if (!have_o) ok = false;
+            }
+            __nv_bfloat16 *orow0 = p.out + (static_cast<size_t>(sg.b) * p.h + head0) * D;
+            if (have_o) {
+                tc_fence_after();
+                float o[NH];
+                tmem_row(tO, o);
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    if (h >= HS) break;
+                    if (whole)
+                        orow0[static_cast<size_t>(h) * D + r] = __float2bfloat16_rn(cres[h] > 0.f ? o[h] / cres[h] : 0.f);
+                    else
+                        slot[static_cast<size_t>(h) * D + r] = o[h];
+                }
+                if (!whole && tid < HS) {
+                    slot[kSpRows * D + tid] = msh[tid];
+                    slot[kSpRows * D + kSpRows + tid] = cres[tid];
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ofree);
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // msh, red and cres are free for the next segment
+            if (c == first_c && tid == 0) p.seg[sidx] = make_int2(first_c, last_c);   // for the merge kernel
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTkTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The merge of the pieces of the segments that were cut between CTAs, in a
+// second launch so that it runs on every SM at once: one block per (segment,
+// head), four warps each folding a quarter of the pieces with the log-sum-exp
+// rule (running max M, sum L, unnormalised O), then warp 0 folds the four.
+
+template <int D>
+__global__ void __launch_bounds__(128)
+    gqa_decode_split_merge_kernel(const float *part, const int2 *seg, __nv_bfloat16 *out, int B, int h, int G,
+                                  int slices, int rows) {
+    constexpr uint32_t SLOT = SplitGeom<D>::kPartFloats;
+    __shared__ float sM[4], sL[4];
+    __shared__ float4 sO[4][D / 4];
+    const int sidx = blockIdx.x, hh = blockIdx.y;
+    const int gs = sidx / B, b = sidx % B;
+    const int g = gs / slices, sl = gs % slices;
+    const int HS = min(G - sl * rows, rows);
+    if (hh >= HS) return;
+    const int2 info = seg[sidx];
+    if (info.x < 0 || info.x == info.y) return;   // an empty sequence, or finished by one CTA
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool act = lane < D / 4;
+    float M = -INFINITY, L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int cc = info.x + warp; cc <= info.y; cc += 4) {
+        const float *sp = part + static_cast<size_t>(cc + sidx) * SLOT;
+        const float m = __ldcg(sp + kSpRows * D + hh);
+        const float l = __ldcg(sp + kSpRows * D + kSpRows + hh);
+        const float4 o = act ? __ldcg(reinterpret_cast<const float4 *>(sp + static_cast<size_t>(hh) * D) + lane)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float M2 = fmaxf(M, m);
+        const float a = M2 == -INFINITY ? 0.f : exp2f(M - M2), w = M2 == -INFINITY ? 0.f : exp2f(m - M2);
+        L = L * a + l * w;
+        acc = make_float4(acc.x * a + o.x * w, acc.y * a + o.y * w, acc.z * a + o.z * w, acc.w * a + o.w * w);
+        M = M2;
+    }
+    if (lane == 0) {
+        sM[warp] = M;
+        sL[warp] = L;
+    }
+    if (act) sO[warp][lane] = acc;
+    __syncthreads();
+    if (warp != 0 || !act) return;
+    float Mf = fmaxf(fmaxf(sM[0], sM[1]), fmaxf(sM[2], sM[3]));
+    float Lf = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int w = 0; w < 4; ++w) {
+        const float wt = sM[w] == -INFINITY ? 0.f : exp2f(sM[w] - Mf);
+        Lf += wt * sL[w];
+        const float4 x = sO[w][lane];
+        o = make_float4(o.x + wt * x.x, o.y + wt * x.y, o.z + wt * x.z, o.w + wt * x.w);
+    }
+    const float inv = Lf > 0.f ? 1.f / Lf : 0.f;
+    __nv_bfloat16 *orow = out + (static_cast<size_t>(b) * h + g * G + sl * rows + hh) * D;
+    *reinterpret_cast<uint2 *>(orow + 4 * lane) =
+        make_uint2(pack_bf16x2(o.x * inv, o.y * inv), pack_bf16x2(o.z * inv, o.w * inv));
+}
+
+// ---------------------------------------------------------------------------
 // host side
 
-static size_t counter_bytes_for(int B, int n_kv, int slices) {
+// bytes of the per-segment records at the start of the workspace (a multiple of 256)
+static size_t seg_bytes_for(int B, int n_kv, int slices) {
     const size_t ns = static_cast<size_t>(n_kv) * slices * B;
-    return (ns * sizeof(int) + 255) & ~static_cast<size_t>(255);
+    return (ns * sizeof(int2) + 255) & ~static_cast<size_t>(255);
 }
 
 template <int D>
 static size_t split_workspace_bytes_t(int B, int n_kv, int slices, int nctas) {
     const size_t ns = static_cast<size_t>(n_kv) * slices * B;
-    return counter_bytes_for(B, n_kv, slices) +
+    return seg_bytes_for(B, n_kv, slices) +
            (static_cast<size_t>(nctas) + ns) * SplitGeom<D>::kPartFloats * sizeof(float);
 }
 
-size_t split_counter_bytes(int B, int h, int n_kv) {
-    const int G = h / n_kv;
-    return counter_bytes_for(B, n_kv, (G + kSpRows - 1) / kSpRows);
-}
 
 size_t split_workspace_bytes(int B, int h, int n_kv, int d) {
     const int G = h / n_kv;
@@ -699,8 +1279,8 @@ static int launch_split_t(const void *q, const void *k, const void *v, long long
     prm.q = static_cast<const __nv_bfloat16 *>(q);
     prm.seqlens = seqlens;
     prm.out = static_cast<__nv_bfloat16 *>(out);
-    prm.count = static_cast<int *>(workspace);
-    prm.part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + counter_bytes_for(B, n_kv, slices));
+    prm.seg = static_cast<int2 *>(workspace);
+    prm.part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + seg_bytes_for(B, n_kv, slices));
     prm.B = B;
     prm.h = h;
     prm.n_kv = n_kv;
@@ -714,12 +1294,82 @@ static int launch_split_t(const void *q, const void *k, const void *v, long long
     if (!prm.status) return 3;
     GQA_SET_TEST_STALL(prm);
     kern<<<nctas, kSpThreads, SG::kTotal, stream>>>(tq, tk, tv, prm);
+    if (cudaGetLastError() != cudaSuccess) return 3;
+    gqa_decode_split_merge_kernel<D><<<dim3(static_cast<unsigned>(n_kv * slices * B), std::min(G, kSpRows)), 128, 0,
+                                       stream>>>(prm.part, prm.seg, prm.out, B, h, G, slices, kSpRows);
+    return cudaGetLastError() == cudaSuccess ? 0 : 3;
+}
+
+// The tokens-as-rows kernel (d = 128, groups of at most 64 heads); the workspace
+// layout and size are those of the heads-as-rows kernel at d = 128.
+template <int NH>
+static int launch_split_tok(const void *q, const void *k, const void *v, long long cache_rows,
+                            const int32_t *seqlens, void *out, int B, int h, int n_kv, float scale, void *workspace,
+                            size_t ws_bytes, cudaStream_t stream) {
+    using TG = TokGeom;
+    auto kern = gqa_decode_split_tok_kernel<NH>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 3;
+    static std::atomic<unsigned long long> attr_done{0};
+    if (!gqa_host::once_per_device(attr_done, dev, [&] {
+            return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TG::kTotal) == cudaSuccess;
+        }))
+        return 3;
+    const int G = h / n_kv;
+    const int nctas = gqa_host::sm_count();
+    if (static_cast<long long>(n_kv) * B > (1LL << 24)) return 2;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+        ws_bytes < split_workspace_bytes_t<128>(B, n_kv, 1, nctas))
+        return 1;
+    CUtensorMap tq, tk, tv;
+    {
+        const uint64_t dims[3] = {128, static_cast<uint64_t>(h), static_cast<uint64_t>(B)};
+        const uint64_t strides[2] = {128 * 2, static_cast<uint64_t>(h) * 128 * 2};
+        const uint32_t box[3] = {64, static_cast<uint32_t>(std::min(NH, h)), 1};
+        if (!gqa_host::encode_tensor_map(&tq, q, 3, dims, strides, box)) return 3;
+    }
+    {
+        const uint64_t dims[3] = {128, static_cast<uint64_t>(n_kv), static_cast<uint64_t>(std::max(cache_rows, 1LL))};
+        const uint64_t strides[2] = {128 * 2, static_cast<uint64_t>(n_kv) * 128 * 2};
+        const uint32_t box[3] = {64, 1, static_cast<uint32_t>(kTkTok)};
+        if (!gqa_host::encode_tensor_map(&tk, k, 3, dims, strides, box)) return 3;
+        if (!gqa_host::encode_tensor_map(&tv, v, 3, dims, strides, box)) return 3;
+    }
+    SplitParams prm = {};
+    prm.q = static_cast<const __nv_bfloat16 *>(q);
+    prm.seqlens = seqlens;
+    prm.out = static_cast<__nv_bfloat16 *>(out);
+    prm.seg = static_cast<int2 *>(workspace);
+    prm.part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + seg_bytes_for(B, n_kv, 1));
+    prm.B = B;
+    prm.h = h;
+    prm.n_kv = n_kv;
+    prm.G = G;
+    prm.slices = 1;
+    prm.nctas = nctas;
+    prm.q_bytes = static_cast<uint32_t>(128 * 2 * std::min(NH, h));
+    prm.cache_rows = cache_rows;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.status = gqa_host::device_status();
+    if (!prm.status) return 3;
+    GQA_SET_TEST_STALL(prm);
+    kern<<<nctas, kSpThreads, TG::kTotal, stream>>>(tq, tk, tv, prm);
+    if (cudaGetLastError() != cudaSuccess) return 3;
+    gqa_decode_split_merge_kernel<128><<<dim3(static_cast<unsigned>(n_kv * B), G), 128, 0, stream>>>(
+        prm.part, prm.seg, prm.out, B, h, G, 1, kTkN);
     return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }
 
 int launch_decode_split(const void *q, const void *k, const void *v, long long cache_rows, const int32_t *seqlens,
                         void *out, int B, int h, int n_kv, int d, float scale, void *workspace, size_t ws_bytes,
                         cudaStream_t stream) {
+    const int G = h / n_kv;
+    if (d == 128 && G <= 16)
+        return launch_split_tok<16>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
+    if (d == 128 && G <= 32)
+        return launch_split_tok<32>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
+    if (d == 128 && G <= 64)
+        return launch_split_tok<64>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
     if (d == 128)
         return launch_split_t<128>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
     return launch_split_t<64>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
@@ -759,8 +1409,6 @@ int launch_decode_split_noalloc(const void *q, const void *k, const void *v, lon
     if (need > kNoAllocScratchBytes) return 1;
     void *scratch = noalloc_scratch();
     if (!scratch) return 3;
-    // the arrival counters must start at zero: clear them on the stream (the rest is scratch)
-    if (cudaMemsetAsync(scratch, 0, split_counter_bytes(B, h, n_kv), stream) != cudaSuccess) return 3;
     return launch_decode_split(q, k, v, cache_rows, seqlens, out, B, h, n_kv, d, scale, scratch, need, stream);
 }
 

@@ -135,16 +135,12 @@ int gqa_decode_rows(const void *q, const void *k_cache, const void *v_cache, int
  *   workspace        DEVICE memory of at least
  *                    gqa_decode_split_workspace_bytes(B, h, n_kv, d_h) bytes
  *                    (which depends on the current device's SM count),
- *                    256-byte aligned, owned by the caller.  Its first
- *                    gqa_decode_split_counter_bytes(B, h, n_kv) bytes are
- *                    arrival counters and must be zero when a call starts;
- *                    every call leaves them zero (also after a wait timed
- *                    out), so a workspace zero-filled once serves any number
- *                    of calls of these sizes.  The rest is scratch.  Before a
- *                    call whose counter bytes exceed those of the earlier
- *                    calls, zero the extra bytes.  Calls that share a
- *                    workspace must not overlap on the GPU (one stream, or
- *                    ordered).
+ *                    256-byte aligned, owned by the caller.  It is scratch:
+ *                    every call writes what it reads, so it needs no
+ *                    initialisation.  Calls that share a workspace must not
+ *                    overlap on the GPU (one stream, or ordered).
+ * The call enqueues two kernels on `stream`: the split decode, then the merge
+ * of the sequences whose tokens fell to several SMs.
  * Errors: as gqa_decode_rows, plus GQA_ERR_INVALID_ARG for a null,
  * misaligned or too small workspace, GQA_ERR_UNSUPPORTED when
  * n_kv * ceil(h / n_kv / 128) * B exceeds 2^24.
@@ -158,10 +154,6 @@ int gqa_decode_split(const void *q, const void *k_cache, const void *v_cache, in
  * device; 0 for sizes gqa_decode_split rejects. */
 size_t gqa_decode_split_workspace_bytes(int B, int h, int n_kv, int d_h);
 
-/* Bytes at the start of the workspace that hold the arrival counters (a
- * multiple of 256); 0 for sizes gqa_decode_split rejects. */
-size_t gqa_decode_split_counter_bytes(int B, int h, int n_kv);
-
 /*
  * gqa_decode_split for callers that may not allocate device memory -- for
  * instance a plug-in running inside another framework that must not touch
@@ -172,9 +164,8 @@ size_t gqa_decode_split_counter_bytes(int B, int h, int n_kv);
  *   Same arguments and result as gqa_decode_split, without the workspace:
  *   the workspace is a fixed 16 MiB array inside the library, which every
  *   device that loads the library holds until the process exits.  The call
- *   allocates nothing (no cudaMalloc, no allocating library routine); it
- *   clears the array's arrival counters with cudaMemsetAsync on `stream`
- *   before the launch.
+ *   allocates nothing (no cudaMalloc, no allocating library routine) and
+ *   needs no clearing (every call writes what it reads).
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture.
@@ -185,8 +176,8 @@ size_t gqa_decode_split_counter_bytes(int B, int h, int n_kv);
  * GQA_ERR_UNSUPPORTED when the sizes need more than the 16 MiB array, that is
  * when gqa_decode_split_workspace_bytes(B, h, n_kv, d_h) exceeds 16 MiB (on a
  * 148-SM B200: n_kv * ceil(h / n_kv / 128) * B above 104 at d_h = 128, above
- * 348 at d_h = 64), and GQA_ERR_CUDA if the address lookup, the clear or the
- * launch fails.  Nothing is launched on an error.
+ * 348 at d_h = 64), and GQA_ERR_CUDA if the address lookup or a launch fails.
+ * Nothing is launched on an argument or size error.
  */
 int gqa_decode_split_noalloc(const void *q, const void *k_cache, const void *v_cache, int64_t cache_rows,
                              const int32_t *seqlens, void *out,

@@ -65,7 +65,7 @@ def test_split_workloads(w):
 def test_split_matches_the_cluster_kernel_and_repeats():
     q, k, v, lens = (t.cuda() for t in inputs.decode_inputs(32, 20, 64, 2, 128, [700] * 10 + [3000] * 10))
     a = gqa.decode_split(q, k, v, lens)
-    b = gqa.decode_split(q, k, v, lens)              # the workspace's counters are back at zero
+    b = gqa.decode_split(q, k, v, lens)              # the same workspace, reused
     c = gqa.gqa_decode_rows                          # the cluster kernel, through its own entry point
     ref = torch.empty_like(q)
     assert c(q.data_ptr(), k.data_ptr(), v.data_ptr(), k.shape[0], lens.data_ptr(), ref.data_ptr(), 20, 64, 2, 128,
@@ -115,13 +115,35 @@ def test_split_lengths_past_the_cache_rows_are_cut_and_reported():
     assert torch.all(got[2] == 0)
 
 
-def test_decode_dispatches_wide_groups_to_the_split_kernel():
-    """decode() sends groups of >= SPLIT_MIN_GROUP heads over caches of >= 256 rows per
-    sequence to gqa_decode_split: the result is bit-identical to calling it directly."""
+def test_decode_dispatch():
+    """decode() sends wide groups, and batches too small to fill the SMs with the cluster
+    kernel's splits, to gqa_decode_split (bit-identical to calling it directly)."""
     G = _lib.SPLIT_MIN_GROUP
     q, k, v, lens = (t.cuda() for t in inputs.decode_inputs(38, 4, G, 1, 128, 2000))
+    assert _lib.use_split(q, k)
     assert torch.equal(gqa.decode(q, k, v, lens), gqa.decode_split(q, k, v, lens))
+    q, k, v, lens = (t.cuda() for t in inputs.decode_inputs(38, 2, 16, 2, 128, 3000))   # 4 units
+    assert _lib.use_split(q, k)
+    assert torch.equal(gqa.decode(q, k, v, lens), gqa.decode_split(q, k, v, lens))
+    q, k, v, lens = (t.cuda() for t in inputs.decode_inputs(38, 16, 64, 8, 128, 300))   # the GQA shape
+    assert not _lib.use_split(q, k)
 
 
 def test_split_status_clean():
     assert gqa.gqa_get_device_status() == _lib.GQA_OK
+
+
+def test_split_running_max_rescales():
+    """Keys along head 0's query, growing every 128 tokens: head 0's running max jumps by
+    more than 2^8 several times inside a CTA's share (the lazy rescale of both kernels)."""
+    for h, n_kv, d in ((32, 1, 128), (64, 2, 64), (256, 1, 128)):
+        q, k, v, lens = inputs.decode_inputs(39 + h, 3, h, n_kv, d, [2000, 700, 5000])
+        k = k.float()
+        off = 0
+        for b in range(3):
+            u = q[b, 0].float() / q[b, 0].float().norm()
+            for j in range(1, min(8, int(lens[b]) // 128)):
+                k[off + 128 * j + 5, 0] = u * (8.0 * j)
+            off += int(lens[b])
+        k = k.to(torch.bfloat16)
+        check(run(q, k, v, lens), oracle.decode(q, k, v, lens), f"split rescales h{h} d{d}", v=v, n_keys=5000)

@@ -150,18 +150,16 @@ def test_product_library_status_clean():
     assert gqa.gqa_get_device_status() == _lib.GQA_OK
 
 
-def test_split_decode_wait_runs_out(W):
-    """The split-KV kernel: the stalled call times out, its workspace counters still
-    return to zero (the next call through the same workspace is exact)."""
-    B, h, n_kv, d = 6, 64, 1, 128
-    q, k, v, L = (t.cuda() for t in inputs.decode_inputs(27, B, h, n_kv, d, [3000, 10, 700, 5000, 64, 1]))
+@pytest.mark.parametrize("B,h,n_kv,d", [(6, 64, 1, 128), (3, 128, 1, 128), (4, 32, 2, 64)], ids=str)
+def test_split_decode_wait_runs_out(W, B, h, n_kv, d):
+    """The split-KV kernels (and their merge): the stalled call times out, and the next
+    call through the same workspace is exact."""
+    q, k, v, L = (t.cuda() for t in inputs.decode_inputs(27, B, h, n_kv, d, [3000, 10, 700, 5000, 64, 1][:B]))
     out = torch.empty_like(q)
     nbytes = W.gqa_decode_split_workspace_bytes(B, h, n_kv, d)
-    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     launch = lambda lib: lib.gqa_decode_split(q.data_ptr(), k.data_ptr(), v.data_ptr(), k.shape[0],  # noqa: E731
                                               L.data_ptr(), out.data_ptr(), B, h, n_kv, d, d ** -0.5,
                                               ws.data_ptr(), nbytes, stream())
     got = stalled_then_clean(W, launch, out)
     assert torch.equal(got, gqa.decode_split(q, k, v, L))
-    counters = ws[:W.gqa_decode_split_counter_bytes(B, h, n_kv)].view(torch.int32)   # at the workspace's start
-    assert torch.all(counters == 0)
