@@ -978,6 +978,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
             // the running max per head (log2 units): msh, copied into registers when they allow
             constexpr bool kMReg = NH <= 32;
             float m[kMReg ? NH : 1];
+#pragma unroll
+            for (int h = 0; h < (kMReg ? NH : 1); ++h) m[h] = -INFINITY;   // set from msh before first use
             auto mv = [&](int h) -> float {
                 if constexpr (kMReg) return m[h];
                 else return msh[h];

@@ -43,8 +43,15 @@
 // the new K/V rows of its own two query tiles into the pages, while the other
 // warps attend.  The attention never reads a slot that is being written:
 // past tiles only cover positions < past.
+//
+// Rows that see few keys (a query tile whose first row sees at most
+// kPfSplitKeys keys) do not average out the bf16 rounding of their softmax
+// weights; for them the weights' bf16 remainders p - bf16(p) are written over
+// the upper half of S as well and multiplied by V in a second product, so the
+// weights are carried to about 16 bits.  That path is a separate
+// instantiation (SPLIT), launched only for the query-tile pairs that need it,
+// so the common path is compiled without it.
 #include <algorithm>
-#include <type_traits>
 
 #include "common.cuh"
 
@@ -61,17 +68,12 @@ constexpr int kPfThreads = 384;  // softmax warpgroups 0 and 1; warpgroup 2 = pr
 constexpr uint32_t kRegsSoftmax = 208, kRegsOther = 80;
 static_assert(256 * kRegsSoftmax + 128 * kRegsOther <= kPfThreads * 168, "register split exceeds the launch");
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-// The softmax weights reach the tensor cores as bf16 (written over S in
-// TMEM).  For a query tile whose first row sees at most this many keys --
-// rows where a few keys can carry most of the weight and the weights'
-// rounding does not average out -- the bf16 remainders p - bf16(p) are also
-// written (over the upper half of S) and multiplied by V in a second product,
-// so those weights are carried to about 16 bits.
-constexpr int kPfSplitKeys = 256;
+constexpr int kPfSplitKeys = 256;            // first-row keys up to which a query tile splits its weights
 
 struct PrefillParams {
     __nv_bfloat16 *out;
-    int B, S_q, S_kv, h, n_kv, G, n_pairs, causal;
+    int B, S_q, S_kv, h, n_kv, G, causal;
+    int pair_lo, pair_hi;          // the query-tile pairs of this launch: [pair_lo, pair_hi)
     float scale_log2;
     int *status;                   // the library's device status word
     // chunked prefill over a paged cache
@@ -106,18 +108,14 @@ __device__ __forceinline__ int chunk_tiles_for(int rows_begin, int S_q, int n_pa
     return n_past + min(rows_begin + kPfRows - 1, S_q - 1) / kPfKeys + 1;
 }
 
-// Whether the weights of the query tile starting at row `row0` go to the
-// tensor cores with their bf16 remainders: its first row (the one that sees
-// the fewest keys) sees at most kPfSplitKeys keys.
-template <bool PAGED>
-__device__ __forceinline__ bool split_weights(const PrefillParams &p, int row0, int past) {
-    const int keys = PAGED ? past + row0 + 1 : p.causal ? min(p.S_kv, row0 + (p.S_kv - p.S_q) + 1) : p.S_kv;
-    return keys <= kPfSplitKeys;
+// The keys the first row of the query tile at row0 sees (the fewest of the tile's rows).
+__host__ __device__ __forceinline__ int first_row_keys(bool paged, int causal, int S_q, int S_kv, int row0,
+                                                       int past) {
+    return paged ? past + row0 + 1 : causal ? min(S_kv, row0 + (S_kv - S_q) + 1) : S_kv;
 }
 
 // The second P V product of a split tile (A = the weights' bf16 remainders in
-// TMEM, B = V): out of line, so the common path of the 80-register MMA issuer
-// keeps its registers.
+// TMEM, B = V): out of line, so the 80-register MMA issuer keeps its registers.
 __device__ __noinline__ void pf_issue_pv_rem(uint32_t d_tmem, uint32_t a_tmem, uint32_t b0, uint32_t lbo,
                                              uint32_t idesc) {
 #pragma unroll
@@ -125,7 +123,7 @@ __device__ __noinline__ void pf_issue_pv_rem(uint32_t d_tmem, uint32_t a_tmem, u
         umma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, lbo, 1024), idesc, 1u);
 }
 
-template <int D, bool PAGED>
+template <int D, bool PAGED, bool SPLIT>
 __global__ void __launch_bounds__(kPfThreads, 1)
     gqa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kp,
@@ -152,7 +150,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int BH = p.B * p.h;
     const int bh = blockIdx.x % BH;
     const int pr = blockIdx.x / BH;
-    const int pair = p.causal ? (p.n_pairs - 1 - pr) : pr;
+    const int pair = p.causal ? (p.pair_hi - 1 - pr) : (p.pair_lo + pr);
     const int b = bh / p.h, head = bh % p.h, kvh = head / p.G;
     const int q0 = pair * 2 * kPfRows;
     // paged chunk: past tokens of this sequence (cut to what the block table can hold)
@@ -313,14 +311,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         umma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, SM::kHalf, 1024), idesc_pv,
                                 (acc || kk > 0) ? 1u : 0u);
                 };
+                // SPLIT: the query tiles whose weights' remainders also multiply V
+                // (tile 0 splits whenever tile 1 does: its rows see fewer keys)
+                int n_split = 0;
+                if constexpr (SPLIT)
+                    n_split = first_row_keys(PAGED, p.causal, p.S_q, p.S_kv, q0 + kPfRows, past) <= kPfSplitKeys ? 2
+                              : first_row_keys(PAGED, p.causal, p.S_q, p.S_kv, q0, past) <= kPfSplitKeys   ? 1
+                                                                                                            : 0;
                 bool ok = mbar_wait(qfull, 0, abort_flag, p.status) && ready(0);
                 if (ok) {
                     if (n_t0 > 0) { issue_qk(0, 0); umma_commit(&sfull[0]); }
                     if (n_t1 > 0) { issue_qk(1, 0); umma_commit(&sfull[1]); }
                     umma_commit(&empty[0]);
                 }
-                // split tiles (tile 0 splits whenever tile 1 does: it sees fewer keys)
-                const int n_split = split_weights<PAGED>(p, q0 + kPfRows, past) ? 2 : split_weights<PAGED>(p, q0, past) ? 1 : 0;
                 for (int j = 0; j < nmax && ok; ++j) {
                     bool v_ready = false, k_next = false;
     #pragma unroll
@@ -345,9 +348,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             }
                         }
                         issue_pv(t, 2 * j + 1, j > 0);
-                        if (t < n_split)   // the remainders: A = the upper half of S
-                            pf_issue_pv_rem(tmem + 256 + t * D, tmem + t * 128 + kPfKeys / 2,
-                                            ring_base + ((2 * j + 1) % kPfRing) * SM::kTile, SM::kHalf, idesc_pv);
+                        if constexpr (SPLIT) {
+                            if (t < n_split)
+                                pf_issue_pv_rem(tmem + 256 + t * D, tmem + t * 128 + kPfKeys / 2,
+                                                ring_base + ((2 * j + 1) % kPfRing) * SM::kTile, SM::kHalf, idesc_pv);
+                        }
                         if (j + 1 < n_t) {
                             if (!k_next) {
                                 if (!ready(2 * j + 2)) { ok = false; continue; }
@@ -403,13 +408,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint32_t tS = tmem + t * 128 + lane_off;
         const uint32_t tO = tmem + 256 + t * D + lane_off;
         const float cl2 = p.scale_log2;
-        const bool split = split_weights<PAGED>(p, q0 + t * kPfRows, past);   // warpgroup-uniform
+        bool split = false;   // (SPLIT only) this tile's weights also go as bf16 remainders; warpgroup-uniform
+        if constexpr (SPLIT)
+            split = first_row_keys(PAGED, p.causal, p.S_q, p.S_kv, q0 + t * kPfRows, past) <= kPfSplitKeys;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        // the key-tile loop, compiled twice: with the weights' bf16 remainders (a split tile)
-        // and without, so the common path carries no extra registers
-        auto tile_loop = [&](auto split_tag) {
-            constexpr bool kSplit = decltype(split_tag)::value;
         for (int j = 0; j < n_t; ++j) {
             const bool landed = mbar_wait(&sfull[t], j & 1, abort_flag, p.status);
             if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }   // tcgen05.ld/st are warp-aligned
@@ -468,30 +471,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     m_used = m_new;
                 }
             }
-            // P = exp2(S * scale * log2(e) - m) as packed bf16, written back over S
-            // (and, for a split tile, the bf16 remainders over the upper half of S);
+            // P = exp2(S * scale * log2(e) - m) as packed bf16, written back over S;
             // the running sum adds exactly the rounded weights P V uses
             float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            // the weights of a key pair (masked keys add nothing, also when scale == 0)
-            auto weights = [&](int c) -> float2 {
-                const float2 x = ffma2_bcast(__uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)), cl2, -m_used);
-                float2 w = make_float2(exp2f(x.x), exp2f(x.y));
-                if (masked) {
-                    if (c > lim_c) w.x = 0.f;
-                    if (c + 1 > lim_c) w.y = 0.f;
-                }
-                return w;
-            };
-            if constexpr (kSplit) {   // the remainders w - bf16(w), exact in fp32, rounded to bf16 (computed
-                                      // first: the main pass below then consumes the S registers as it goes)
+            if (SPLIT && split) {   // first the remainders w - bf16(w) (exact in fp32), as bf16, over
+                                    // the upper half of S (its scores are in registers already)
 #pragma unroll
                 for (int ch = 0; ch < kPfKeys / 16; ++ch) {
                     uint32_t rk[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float2 w = weights(ch * 16 + 2 * e);
-                        const float2 u = unpack_bf16x2(pack_bf16x2(w.x, w.y));
-                        rk[e] = pack_bf16x2(w.x - u.x, w.y - u.y);
+                        const int c = ch * 16 + 2 * e;
+                        const float2 x =
+                            ffma2_bcast(__uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)), cl2, -m_used);
+                        float w0 = exp2f(x.x), w1 = exp2f(x.y);
+                        if (masked) {
+                            if (c > lim_c) w0 = 0.f;
+                            if (c + 1 > lim_c) w1 = 0.f;
+                        }
+                        const float2 u = unpack_bf16x2(pack_bf16x2(w0, w1));
+                        rk[e] = pack_bf16x2(w0 - u.x, w1 - u.y);
                         rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(rk[e]));
                     }
                     tmem_st8(tS + kPfKeys / 2 + ch * 8, rk);
@@ -502,9 +501,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float2 w = weights(ch * 32 + 2 * e);
-                    pk[e] = pack_bf16x2(w.x, w.y);
-                    rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(pk[e]));
+                    const int c = ch * 32 + 2 * e;
+                    const float2 x = ffma2_bcast(__uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)), cl2, -m_used);
+                    uint32_t pp = pack_bf16x2(exp2f(x.x), exp2f(x.y));
+                    if (masked) {   // masked keys add nothing (also when scale == 0)
+                        if (c > lim_c) pp &= 0xFFFF0000u;
+                        if (c + 1 > lim_c) pp &= 0x0000FFFFu;
+                    }
+                    pk[e] = pp;
+                    rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(pp));
                 }
                 tmem_st16(tS + ch * 16, pk);
             }
@@ -515,11 +520,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tc_fence_before();
             mbar_arrive(&pfull[t]);
         }
-        };
-        if (split)
-            tile_loop(std::true_type{});
-        else
-            tile_loop(std::false_type{});
         // epilogue: O / l -> bf16 -> out[b, row, head, :]
         const bool fin = n_t > 0 && ok && mbar_wait(&odone[t], 0, abort_flag, p.status);
         if (__all_sync(0xffffffffu, fin)) {
@@ -568,10 +568,10 @@ struct PrefillCall {
     int max_blocks, page_size, num_pages;
 };
 
-template <int D, bool PAGED>
-static int launch_prefill_t(const PrefillCall &c) {
+template <int D, bool PAGED, bool SPLIT>
+static int launch_prefill_range(const PrefillCall &c, int pair_lo, int pair_hi) {
     using SM = PrefillSmem<D>;
-    auto kern = gqa_prefill_kernel<D, PAGED>;
+    auto kern = gqa_prefill_kernel<D, PAGED, SPLIT>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 3;
     static std::atomic<unsigned long long> attr_done{0};
@@ -618,7 +618,8 @@ static int launch_prefill_t(const PrefillCall &c) {
     prm.h = c.h;
     prm.n_kv = c.n_kv;
     prm.G = c.h / c.n_kv;
-    prm.n_pairs = (c.S_q + 2 * kPfRows - 1) / (2 * kPfRows);
+    prm.pair_lo = pair_lo;
+    prm.pair_hi = pair_hi;
     prm.causal = c.causal ? 1 : 0;
     prm.scale_log2 = c.scale * 1.4426950408889634f;
     prm.status = gqa_host::device_status();
@@ -633,10 +634,31 @@ static int launch_prefill_t(const PrefillCall &c) {
     prm.max_blocks = c.max_blocks;
     prm.page_size = c.page_size;
     prm.num_pages = c.num_pages;
-    const long ctas = static_cast<long>(prm.n_pairs) * c.B * c.h;
+    const long ctas = static_cast<long>(pair_hi - pair_lo) * c.B * c.h;
+    if (ctas <= 0) return 0;
     if (ctas > 0x7fffffffL) return 1;
     kern<<<static_cast<unsigned>(ctas), kPfThreads, SM::kTotal, c.stream>>>(tq, tk, tv, tkp, tvp, prm);
     return cudaGetLastError() == cudaSuccess ? 0 : 3;
+}
+
+// The pairs whose first query tile splits its weights go to the SPLIT instantiation
+// (pairs [0, n_sp): the keys a tile's first row sees grow with the pair), the rest to
+// the common one.  The chunked prefill (PAGED) cannot tell on the host (the past
+// lengths live on the device): it runs the SPLIT instantiation, which decides per tile.
+template <int D, bool PAGED>
+static int launch_prefill_t(const PrefillCall &c) {
+    const int n_pairs = (c.S_q + 2 * kPfRows - 1) / (2 * kPfRows);
+    if constexpr (PAGED) {
+        return launch_prefill_range<D, true, true>(c, 0, n_pairs);
+    } else {
+        int n_sp = 0;
+        while (n_sp < n_pairs &&
+               first_row_keys(false, c.causal, c.S_q, c.S_kv, n_sp * 2 * kPfRows, 0) <= kPfSplitKeys)
+            ++n_sp;
+        int st = launch_prefill_range<D, false, false>(c, n_sp, n_pairs);
+        if (st == 0) st = launch_prefill_range<D, false, true>(c, 0, n_sp);
+        return st;
+    }
 }
 
 int launch_prefill(const void *q, const void *k, const void *v, void *out, int B, int S_q, int S_kv, int h, int n_kv,
