@@ -13,12 +13,17 @@
 // and more heads the warp-level mma.sync path of the cluster decode kernel
 // cannot keep up with HBM; and with ragged lengths a fixed number of splits
 // per sequence leaves most SMs idle while the longest sequences finish.  Here:
-//   - the G heads of a group are the M = 128 rows of tcgen05 MMAs (padded),
-//     the stage's 64 tokens the N columns: S = Q K^T lands in TMEM, one
-//     softmax thread per head row turns it into P (bf16, written back over
-//     S), and O += P V accumulates in TMEM (A = P from TMEM, B = V from shared
-//     memory), exactly the structure of the prefill kernel with the heads of
-//     one token in place of the query rows of one head;
+//   - the G heads of a group are the M = 128 rows of tcgen05 MMAs, the
+//     stage's 64 tokens the N columns: S = Q K^T lands in TMEM (A = Q, held
+//     in TMEM; B = K from shared memory), one softmax thread per row turns it
+//     into P (bf16, written back over S), and O += P V accumulates in TMEM
+//     (A = P from TMEM, B = V from shared memory): the structure of the
+//     prefill kernel with the heads of one token in place of the query rows
+//     of one head.  A group of at most 64 (32) heads fills the 128 rows with
+//     2 (4) copies of its queries; copy k takes its own quarter (half) of
+//     every stage's tokens, with its own running max and sum, and the
+//     segment's epilogue merges the copies (log-sum-exp, through shared
+//     memory), so all four softmax warps work whatever the group size;
 //   - work = (KV head, head slice, sequence, token); the batch's tokens of
 //     every (KV head, slice) are laid end to end and CTA c of the persistent
 //     grid (one per SM) takes the range [c W / NC, (c + 1) W / NC), whatever
@@ -28,11 +33,13 @@
 //     max, running sum, unnormalised O) in the caller's workspace, and a
 //     second, small kernel merges them with the log-sum-exp rule, one block
 //     per (segment, head) on every SM at once;
-//   - roles: warp 4 streams Q (once per segment) and K/V stages with TMA into
-//     a ring, warp 5 allocates TMEM and issues the MMAs, warps 0-3 run the
-//     softmax (lazy rescale: the running max moves only when a row's stage
-//     max exceeds it by 2^8) and the epilogue.  S is double-buffered in TMEM,
-//     so Q K^T of stage i + 1 runs while the softmax of stage i does.
+//   - roles: warp 4 streams the K/V stages with TMA into a ring, warp 5
+//     allocates TMEM and issues the MMAs, warps 0-3 write each segment's Q
+//     into TMEM (the next segment's as soon as the last S of the current one
+//     is read), run the softmax (lazy rescale: the running max moves only
+//     when a row's stage max exceeds it by 2^8) and the epilogue.  S is
+//     double-buffered in TMEM, so Q K^T of stage i + 1 runs while the
+//     softmax of stage i does.
 // Workspace: one record per segment first (the CTAs of its first and last
 // piece, written by the CTA of the first piece; (-1, -1) for an empty
 // sequence), padded to 256 bytes, then the partial slots (CTA c's piece of
@@ -47,24 +54,25 @@
 
 namespace gqa {
 
-constexpr int kSpRows = 128;                 // MMA M: query heads of one KV group (padded)
+constexpr int kSpRows = 128;                 // MMA M: query heads of one KV group (padded, or replicated)
 constexpr int kSpTok = 64;                   // tokens per stage (N of S = Q K^T, K of O += P V)
 constexpr int kSpThreads = 192;              // warps 0-3 softmax + epilogue, 4 producer, 5 MMA
 constexpr int kSpRingBytes = 192 * 1024;     // K/V ring
 constexpr float kSpRescale = 8.0f;           // lazy rescale threshold (log2 units)
 constexpr int kSpSplitAllBelow = 256;        // sequences this short also send the weights' bf16 remainders
-constexpr uint32_t kSpTmemCols = 256;        // S0 [0, 64), S1 [64, 128), O [128, 128 + D)
+constexpr uint32_t kSpTmemCols = 512;        // S0 [0, 64), S1 [64, 128), O [128, 128 + D), Q [256, 256 + D / 2)
+constexpr uint32_t kSpQCol = 256;
+constexpr int kSpMrgStride = 36;             // floats per row of the replica-merge buffer (32 + 4: no bank conflicts)
 
 template <int D>
 struct SplitGeom {
-    static constexpr uint32_t kQ = kSpRows * D * 2;     // Q tile: D / 64 panels of 128 rows x 128 bytes
-    static constexpr uint32_t kQPanel = kSpRows * 128;
     static constexpr uint32_t kKV = kSpTok * D * 2;     // K (or V) of a stage: D / 64 panels of 64 rows x 128 B
     static constexpr uint32_t kKVPanel = kSpTok * 128;
     static constexpr uint32_t kSlot = 2 * kKV;
     static constexpr int kRing = kSpRingBytes / kSlot;  // 6 (D = 128) or 12 (D = 64)
     static constexpr uint32_t kCtrl = 512;
-    static constexpr uint32_t kTotal = kQ + kRing * kSlot + kCtrl + 1024;
+    static constexpr uint32_t kMerge = (kSpRows * kSpMrgStride + 2 * kSpRows) * 4;   // replica merge: O chunk, m, l
+    static constexpr uint32_t kTotal = kRing * kSlot + kCtrl + kMerge + 1024;
     static constexpr uint32_t kPartFloats = kSpRows * D + 2 * kSpRows;   // one partial slot: O, m, l
     static_assert(kRing >= 3, "the ring must hold the stage being multiplied and two ahead");
 };
@@ -142,22 +150,44 @@ __device__ __forceinline__ int split_owner(long long w, long long W, int nc) {
     return static_cast<int>(((w + 1) * nc - 1) / W);
 }
 
-template <int D>
+// bar.red.and over the first n threads of the block on named barrier id: true iff
+// pred holds in every one of them
+__device__ __forceinline__ bool bar_red_and(int id, int n, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+// GP = rows of one copy of the group's heads: 128 (groups of more than 64 heads, in
+// slices of 128), 64 or 32.  With GP < 128 the 128 MMA rows hold 128 / GP copies of
+// the group's queries, and copy k takes columns [k TPR, (k + 1) TPR) of every stage
+// (TPR = 64 GP / 128 tokens): each copy keeps its own running max, sum and O rows,
+// over its share of the tokens (its weights for the other copies' tokens are zero),
+// and the epilogue merges the copies with the log-sum-exp rule.  So all four softmax
+// warps share every stage whatever the group size, and each thread exponentiates
+// TPR scores instead of 64.
+template <int D, int GP>
 __global__ void __launch_bounds__(kSpThreads, 1)
-    gqa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                            const __grid_constant__ CUtensorMap tm_v, const SplitParams p) {
+    gqa_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                            const SplitParams p) {
     using SG = SplitGeom<D>;
-    constexpr int R = SG::kRing;
+    constexpr int NR = SG::kRing;
+    constexpr int REP = kSpRows / GP;       // copies of the group's queries down the MMA rows
+    constexpr int TPR = kSpTok / REP;       // stage columns of one copy
+    static_assert(GP == 32 || GP == 64 || GP == 128, "one copy spans whole warps");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sQ = smem;
-    uint8_t *sRing = smem + SG::kQ;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sRing + R * SG::kSlot);
-    uint64_t *qfull = bars;               // Q of the segment landed
-    uint64_t *qfree = qfull + 1;          // the segment's last Q K^T is done (Q may be replaced)
-    uint64_t *full = qfree + 1;           // [R] stage landed
-    uint64_t *empty = full + R;           // [R] stage's P V done
-    uint64_t *sfull = empty + R;          // [2] S buffer written
+    uint8_t *sRing = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sRing + NR * SG::kSlot);
+    uint64_t *qfull = bars;               // the segment's Q is in TMEM (one arrival per softmax warp)
+    uint64_t *full = qfull + 1;           // [NR] stage landed
+    uint64_t *empty = full + NR;          // [NR] stage's P V done
+    uint64_t *sfull = empty + NR;         // [2] S buffer written
     uint64_t *pfull = sfull + 2;          // [2] P written over the S buffer (one arrival per softmax warp)
     // [2] P V of stage gi completes phase gi / 2 of pvdone[gi % 2].  Two barriers, because a
     // parity wait only tells the latest phase from the one before it: the softmax waits for
@@ -169,14 +199,16 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     long long *scan = reinterpret_cast<long long *>(drain + 2);   // [8]: block-scan scratch (after tmem/abort)
+    float *mrg = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + SG::kCtrl);   // [128][36]
+    float *mrg_m = mrg + kSpRows * kSpMrgStride;                  // [128]
+    float *mrg_l = mrg_m + kSpRows;                               // [128]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = blockIdx.x, NC = p.nctas;
 
     if (threadIdx.x == 0) {
-        mbar_init(qfull, 1);
-        mbar_init(qfree, 1);
-        for (int i = 0; i < R; ++i) {
+        mbar_init(qfull, 4);
+        for (int i = 0; i < NR; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
@@ -281,25 +313,18 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     if (warp == 4) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             SplitCursor cu = cursor();
             SplitSeg sg;
-            int gi = 0, seg = 0;
+            int gi = 0;
             const int first_loaded = GQA_STALLED(p) ? 1 : 0;   // wait-test build: stage 0 never arrives
             bool ok = true;
             while (ok && cu.next(sg)) {
-                const int g = sg.gs / p.slices, sl = sg.gs % p.slices;
-                const int head0 = g * p.G + sl * kSpRows;
-                if (seg > 0 && !mbar_wait(qfree, (seg - 1) & 1, abort_flag, p.status)) break;
-                mbar_arrive_expect_tx(qfull, p.q_bytes);
-                for (int hf = 0; hf < D / 64; ++hf)
-                    tma_load_3d(sQ + hf * SG::kQPanel, &tm_q, qfull, hf * 64, head0, sg.b);
-                ++seg;   // Q loads issued
+                const int g = sg.gs / p.slices;
                 const int n = n_stages(sg);
                 for (int i = 0; i < n; ++i, ++gi) {
-                    const int slot = gi % R, use = gi / R;
+                    const int slot = gi % NR, use = gi / NR;
                     if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, abort_flag, p.status)) {
                         ok = false;
                         break;
@@ -315,9 +340,8 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                 }
             }
             if (*abort_flag) {   // let the copies in flight land before the CTA moves on
-                if (seg > 0) mbar_wait_drain(qfull, (seg - 1) & 1, p.status);
-                for (int i = max(first_loaded, gi - R); i < gi; ++i)
-                    mbar_wait_drain(&full[i % R], (i / R) & 1, p.status);
+                for (int i = max(first_loaded, gi - NR); i < gi; ++i)
+                    mbar_wait_drain(&full[i % NR], (i / NR) & 1, p.status);
             }
         }
         __syncwarp();
@@ -325,28 +349,34 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         // ------------------------------------------------------------ MMA issuer (warp-wide loop, lane 0 issues)
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kSpRows, kSpTok, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(kSpRows, D, false, true);
-        const uint32_t q_base = smem_u32(sQ);
         const uint32_t ring_base = smem_u32(sRing);
         auto wait1 = [&](uint64_t *bar, uint32_t parity) -> bool {   // lane 0 waits, the warp learns the outcome
             int r = 1;
             if (lane == 0) r = mbar_wait(bar, parity, abort_flag, p.status);
             return __shfl_sync(0xffffffffu, r, 0) != 0;
         };
-        auto issue_qk = [&](int gi) {   // S[gi % 2] = Q K(stage gi)^T
+        auto issue_qk = [&](int gi) {   // S[gi % 2] = Q K(stage gi)^T, A = Q from TMEM
             const uint32_t d_tmem = tmem + (gi & 1) * kSpTok;
-            const uint32_t b0 = ring_base + (gi % R) * SG::kSlot;
+            const uint32_t b0 = ring_base + (gi % NR) * SG::kSlot;
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks)
-                umma_ss(d_tmem, sdesc_sw128(q_base + (ks >> 2) * SG::kQPanel + (ks & 3) * 32, 16, 1024),
-                        sdesc_sw128(b0 + (ks >> 2) * SG::kKVPanel + (ks & 3) * 32, 16, 1024), idesc_qk, ks > 0);
+                umma_ts(d_tmem, tmem + kSpQCol + ks * 8,
+                        sdesc_sw128(b0 + (ks >> 2) * SG::kKVPanel + (ks & 3) * 32, 16, 1024), idesc_qk,
+                        ks > 0 ? 1u : 0u);
         };
         auto issue_pv = [&](int gi, bool acc, bool rem) {   // O (+)= P[gi % 2] V(stage gi); rem: the remainders
             const uint32_t a_tmem = tmem + (gi & 1) * kSpTok + (rem ? kSpTok / 2 : 0);
-            const uint32_t b0 = ring_base + (gi % R) * SG::kSlot + SG::kKV;
+            const uint32_t b0 = ring_base + (gi % NR) * SG::kSlot + SG::kKV;
 #pragma unroll
             for (int kk = 0; kk < kSpTok / 16; ++kk)
                 umma_ts(tmem + 2 * kSpTok, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, SG::kKVPanel, 1024),
                         idesc_pv, (acc || rem || kk > 0) ? 1u : 0u);
+        };
+        // lane 0 tests a barrier without blocking, the warp learns the outcome
+        auto test1 = [&](uint64_t *bar, uint32_t parity) -> bool {
+            int r = 0;
+            if (lane == 0) r = mbar_try_wait(bar, parity);
+            return __shfl_sync(0xffffffffu, r, 0) != 0;
         };
         SplitCursor cu = cursor();
         SplitSeg sg;
@@ -356,56 +386,76 @@ __global__ void __launch_bounds__(kSpThreads, 1)
             const int n = n_stages(sg);
             const bool split = sg.L <= kSpSplitAllBelow;
             ok = wait1(qfull, seg & 1);
-            // Q K^T of the first two stages
-            for (int i = 0; i < min(n, 2) && ok; ++i) {
-                ok = wait1(&full[(gi0 + i) % R], ((gi0 + i) / R) & 1);
-                if (!ok) break;
-                tc_fence_after();
-                if (lane == 0) {
-                    issue_qk(gi0 + i);
-                    umma_commit(&sfull[(gi0 + i) & 1]);
-                    if (i == n - 1) umma_commit(qfree);
-                }
-                __syncwarp();
-            }
-            for (int i = 0; i < n && ok; ++i) {
-                const int gi = gi0 + i;
-                ok = wait1(&pfull[gi & 1], (gi >> 1) & 1);
-                if (ok && i == 0 && seg > 0) ok = wait1(ofree, (seg - 1) & 1);   // the last segment's O is read out
-                if (!ok) break;
-                tc_fence_after();
-                const int valid = min(kSpTok, sg.t1 - (sg.t0 + i * kSpTok));
-                if (valid < kSpTok) {
-                    // the stage runs past the segment: its V rows there belong to other CTAs or
-                    // other sequences (or read as zeros); clear them so that 0 * (whatever they
-                    // hold) adds nothing
-                    uint8_t *vt = sRing + (gi % R) * SG::kSlot + SG::kKV;
-                    for (int hf = 0; hf < D / 64; ++hf)
-                        for (int it = lane; it < (kSpTok - valid) * 8; it += 32) {
-                            const int r = valid + it / 8, ch = it % 8;
-                            *reinterpret_cast<uint4 *>(vt + hf * SG::kKVPanel + r * 128 + ch * 16) =
-                                make_uint4(0u, 0u, 0u, 0u);
+            // Issue Q K^T(nq) once its stage has landed and P V(nq - 2) is issued (S buffer
+            // nq % 2 is free), and P V(np) once its P is written -- whichever is ready first,
+            // so that a stage still in flight does not hold back the P V (and the ring slot
+            // it frees) of one that is done.  Gives up like mbar_wait when nothing moves.
+            int nq = 0, np = 0;
+            bool ofree_ok = seg == 0;
+            uint32_t idle = 0;
+            unsigned long long t_idle = 0;
+            while (ok && np < n) {
+                bool moved = false;
+                if (np < nq) {
+                    const int gi = gi0 + np;
+                    if (!ofree_ok) ofree_ok = test1(ofree, (seg - 1) & 1);   // the last segment's O is read out
+                    if (ofree_ok && test1(&pfull[gi & 1], (gi >> 1) & 1)) {
+                        tc_fence_after();
+                        const int valid = min(kSpTok, sg.t1 - (sg.t0 + np * kSpTok));
+                        if (valid < kSpTok) {
+                            // the stage runs past the segment: its V rows there belong to other CTAs or
+                            // other sequences (or read as zeros); clear them so that 0 * (whatever they
+                            // hold) adds nothing
+                            uint8_t *vt = sRing + (gi % NR) * SG::kSlot + SG::kKV;
+                            for (int hf = 0; hf < D / 64; ++hf)
+                                for (int it = lane; it < (kSpTok - valid) * 8; it += 32) {
+                                    const int r = valid + it / 8, ch = it % 8;
+                                    *reinterpret_cast<uint4 *>(vt + hf * SG::kKVPanel + r * 128 + ch * 16) =
+                                        make_uint4(0u, 0u, 0u, 0u);
+                                }
+                            fence_proxy_async_smem();   // generic-proxy stores before the tensor core reads
+                            __syncwarp();
                         }
-                    fence_proxy_async_smem();   // generic-proxy stores before the tensor core reads
-                    __syncwarp();
-                }
-                if (lane == 0) {
-                    issue_pv(gi, i > 0, false);
-                    if (split) issue_pv(gi, true, true);
-                    umma_commit(&empty[gi % R]);
-                    umma_commit(&pvdone[gi & 1]);
-                }
-                __syncwarp();
-                if (i + 2 < n) {
-                    ok = wait1(&full[(gi + 2) % R], ((gi + 2) / R) & 1);
-                    if (!ok) break;
-                    tc_fence_after();
-                    if (lane == 0) {
-                        issue_qk(gi + 2);
-                        umma_commit(&sfull[gi & 1]);
-                        if (i + 2 == n - 1) umma_commit(qfree);
+                        if (lane == 0) {
+                            issue_pv(gi, np > 0, false);
+                            if (split) issue_pv(gi, true, true);
+                            umma_commit(&empty[gi % NR]);
+                            umma_commit(&pvdone[gi & 1]);
+                        }
+                        __syncwarp();
+                        ++np;
+                        moved = true;
                     }
-                    __syncwarp();
+                }
+                if (nq < n && nq <= np + 1) {
+                    const int gi = gi0 + nq;
+                    if (test1(&full[gi % NR], (gi / NR) & 1)) {
+                        tc_fence_after();
+                        if (lane == 0) {
+                            issue_qk(gi);
+                            umma_commit(&sfull[gi & 1]);
+                        }
+                        __syncwarp();
+                        ++nq;
+                        moved = true;
+                    }
+                }
+                if (moved) {
+                    idle = 0;
+                } else if (++idle == 1) {
+                    t_idle = global_ns();
+                } else if ((idle & 63u) == 0) {
+                    int give_up = 0;
+                    if (lane == 0) {
+                        if (*abort_flag) {
+                            give_up = 1;
+                        } else if (global_ns() - t_idle > kWaitLimitNs) {
+                            record_timeout(p.status);
+                            *abort_flag = 1;
+                            give_up = 1;
+                        }
+                    }
+                    if (__shfl_sync(0xffffffffu, give_up, 0)) ok = false;
                 }
             }
             gi0 += n;
@@ -417,19 +467,75 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax + epilogue (warps 0-3, row = head)
-        const int r = warp * 32 + lane;                                  // TMEM lane = head row of the tile
+        // ------------------------------------------------------------ softmax + epilogue (warps 0-3)
+        // thread r = TMEM lane r = row r: head hr of copy kr, which owns stage columns [c0, c0 + TPR)
+        const int r = warp * 32 + lane;
+        const int kr = r / GP, hr = r % GP;            // kr is warp-uniform
+        const int c0 = kr * TPR;
         const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
         const uint32_t tO = tmem + 2 * kSpTok + lane_off;
+        // Q of a segment into TMEM (row r = head hr of the slice; rows past the group's heads are zero)
+        auto write_q = [&](const SplitSeg &s) {
+            const int g = s.gs / p.slices, sl = s.gs % p.slices;
+            const int HS = min(p.G - sl * kSpRows, GP);
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                p.q + (static_cast<size_t>(s.b) * p.h + g * p.G + sl * kSpRows + (hr < HS ? hr : 0)) * D);
+#pragma unroll
+            for (int half = 0; half < D / 64; ++half) {
+                uint32_t x[32];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const uint4 v = hr < HS ? src[half * 8 + e] : make_uint4(0u, 0u, 0u, 0u);
+                    x[4 * e] = v.x;
+                    x[4 * e + 1] = v.y;
+                    x[4 * e + 2] = v.z;
+                    x[4 * e + 3] = v.w;
+                }
+                tmem_st32(tmem + kSpQCol + half * 32 + lane_off, x);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(qfull);
+        };
+        // this thread's packed weights (TPR / 2 columns from c0 / 2) and zeros in the other
+        // copies' columns, over columns [base, base + 32) of its S row
+        auto put_p = [&](uint32_t tS, uint32_t base, const uint32_t (&pk)[TPR / 2]) {
+            if constexpr (REP == 1) {
+                uint32_t a[16], b2[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    a[e] = pk[e];
+                    b2[e] = pk[16 + e];
+                }
+                tmem_st16(tS + base, a);
+                tmem_st16(tS + base + 16, b2);
+            } else if constexpr (REP == 2) {
+                uint32_t z[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) z[e] = 0u;
+                tmem_st16(tS + base + c0 / 2, pk);
+                tmem_st16(tS + base + (16 - c0 / 2), z);
+            } else {
+                uint32_t z[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) z[e] = 0u;
+                tmem_st8(tS + base + c0 / 2, pk);
+#pragma unroll
+                for (int k = 1; k < REP; ++k) tmem_st8(tS + base + ((kr + k) % REP) * 8, z);
+            }
+        };
         SplitCursor cu = cursor();
         SplitSeg sg;
         int gi0 = 0, seg = 0;
         bool ok = true;
-        while (cu.next(sg)) {
+        bool have = cu.next(sg);
+        if (have) write_q(sg);
+        while (have) {
             const int g = sg.gs / p.slices, sl = sg.gs % p.slices;
             const int head0 = g * p.G + sl * kSpRows;
-            const int HS = min(p.G - sl * kSpRows, kSpRows);
-            const bool live = warp * 32 < HS;                            // this warp holds real heads
+            const int HS = min(p.G - sl * kSpRows, GP);
+            const bool live = REP > 1 || warp * 32 < HS;                 // this warp holds real heads
             const int n = n_stages(sg);
             const bool split = sg.L <= kSpSplitAllBelow;
             float m_used = -INFINITY, l = 0.f;
@@ -443,18 +549,32 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                 }
                 tc_fence_after();
                 if (live) {
-                    const int valid = min(kSpTok, sg.t1 - (sg.t0 + i * kSpTok));   // columns < valid are tokens
-                    uint32_t s0[32], s1[32];
-                    tmem_ld32(tS, s0);
-                    tmem_ld32(tS + 32, s1);
+                    // columns c0 + j, j < vm, are tokens of the segment (vm may be <= 0 for a copy
+                    // whose share of the segment's last stage is empty)
+                    const int vm = min(kSpTok, sg.t1 - (sg.t0 + i * kSpTok)) - c0;
+                    uint32_t s[TPR];
+                    if constexpr (TPR == 16) {
+                        tmem_ld16(tS + c0, s);
+                    } else if constexpr (TPR == 32) {
+                        tmem_ld32(tS + c0, s);
+                    } else {
+                        uint32_t s0[32], s1[32];
+                        tmem_ld32(tS, s0);
+                        tmem_ld32(tS + 32, s1);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            s[j] = s0[j];
+                            s[32 + j] = s1[j];
+                        }
+                    }
                     tmem_wait_ld();
-#define GQA_SP(cc) ((cc) < 32 ? s0[(cc)] : s1[(cc) - 32])
                     float mx = -INFINITY;
 #pragma unroll
-                    for (int cc = 0; cc < kSpTok; cc += 2)
-                        mx = fmax3(mx, cc < valid ? __uint_as_float(GQA_SP(cc)) : -INFINITY,
-                                   cc + 1 < valid ? __uint_as_float(GQA_SP(cc + 1)) : -INFINITY);
-                    const float m_tile = mx * cl2;   // >= 1 valid token per stage
+                    for (int j = 0; j < TPR; j += 2)
+                        mx = fmax3(mx, j < vm ? __uint_as_float(s[j]) : -INFINITY,
+                                   j + 1 < vm ? __uint_as_float(s[j + 1]) : -INFINITY);
+                    const float m_tile = mx == -INFINITY ? -INFINITY : mx * cl2;
                     if (i == 0) {
                         m_used = m_tile;
                     } else {
@@ -469,7 +589,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                             }
                             tc_fence_after();
                             const float m_new = need ? m_tile : m_used;
-                            const float alpha = exp2f(m_used - m_new);
+                            const float alpha = exp2f(m_used - m_new);   // 0 while m_used is -inf
 #pragma unroll
                             for (int cc = 0; cc < D / 32; ++cc) {
                                 uint32_t ro[32];
@@ -485,45 +605,31 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                         }
                     }
                     float2 rs = make_float2(0.f, 0.f);
-                    auto weights = [&](int cc) -> float2 {
-                        const float2 x = ffma2_bcast(__uint_as_float(GQA_SP(cc)), __uint_as_float(GQA_SP(cc + 1)),
-                                                     cl2, -m_used);
+                    auto weights = [&](int j) -> float2 {
+                        const float2 x = ffma2_bcast(__uint_as_float(s[j]), __uint_as_float(s[j + 1]), cl2, -m_used);
                         float2 w = make_float2(exp2f(x.x), exp2f(x.y));
-                        if (cc >= valid) w.x = 0.f;   // columns past the segment's tokens add nothing
-                        if (cc + 1 >= valid) w.y = 0.f;
+                        if (j >= vm) w.x = 0.f;   // columns past the segment's tokens add nothing
+                        if (j + 1 >= vm) w.y = 0.f;
                         return w;
                     };
-                    if (split) {   // the bf16 remainders w - bf16(w) over the upper half of S
-                        uint32_t rk[16];
+                    uint32_t pk[TPR / 2];
+                    if (split) {   // the bf16 remainders w - bf16(w), over the upper half of S
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) {
+                        for (int e = 0; e < TPR / 2; ++e) {
                             const float2 w = weights(2 * e);
                             const float2 u = unpack_bf16x2(pack_bf16x2(w.x, w.y));
-                            rk[e] = pack_bf16x2(w.x - u.x, w.y - u.y);
-                            rs = fadd2(rs, unpack_bf16x2(rk[e]));
-                        }
-                        tmem_st16(tS + kSpTok / 2, rk);
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float2 w = weights(32 + 2 * e);
-                            const float2 u = unpack_bf16x2(pack_bf16x2(w.x, w.y));
-                            rk[e] = pack_bf16x2(w.x - u.x, w.y - u.y);
-                            rs = fadd2(rs, unpack_bf16x2(rk[e]));
-                        }
-                        tmem_st16(tS + kSpTok / 2 + 16, rk);
-                    }
-#pragma unroll
-                    for (int ch = 0; ch < kSpTok / 32; ++ch) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float2 w = weights(ch * 32 + 2 * e);
-                            pk[e] = pack_bf16x2(w.x, w.y);
+                            pk[e] = pack_bf16x2(w.x - u.x, w.y - u.y);
                             rs = fadd2(rs, unpack_bf16x2(pk[e]));
                         }
-                        tmem_st16(tS + ch * 16, pk);
+                        put_p(tS, kSpTok / 2, pk);
                     }
-#undef GQA_SP
+#pragma unroll
+                    for (int e = 0; e < TPR / 2; ++e) {
+                        const float2 w = weights(2 * e);
+                        pk[e] = pack_bf16x2(w.x, w.y);
+                        rs = fadd2(rs, unpack_bf16x2(pk[e]));
+                    }
+                    put_p(tS, 0, pk);
                     l += rs.x + rs.y;
                     tmem_wait_st();
                 }
@@ -532,11 +638,15 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                 if (lane == 0) mbar_arrive(&pfull[gi & 1]);
             }
             gi0 += n;
+            const SplitSeg cur = sg;
+            have = cu.next(sg);
+            // the next segment's Q: every Q K^T of this one is done (its S were all read above)
+            if (have && ok) write_q(sg);
 
             // ---- epilogue of the segment: O / l directly, or a partial result and the merge
-            const int first_c = split_owner(sg.w, W, NCe), last_c = split_owner(sg.w + sg.L - 1, W, NCe);
+            const int first_c = split_owner(cur.w, W, NCe), last_c = split_owner(cur.w + cur.L - 1, W, NCe);
             const bool whole = first_c == last_c;
-            const int sidx = sg.gs * p.B + sg.b;
+            const int sidx = cur.gs * p.B + cur.b;
             float *slot = p.part + static_cast<size_t>(c + sidx) * SG::kPartFloats;
             bool have_o = false;
             if (ok) {
@@ -544,34 +654,116 @@ __global__ void __launch_bounds__(kSpThreads, 1)
                 have_o = __all_sync(0xffffffffu, fin);
                 if (!have_o) ok = false;
             }
-            if (have_o && live) {
-                tc_fence_after();
-                const bool row_ok = r < HS;
-                const float inv = 1.f / l;
-                __nv_bfloat16 *orow = p.out + (static_cast<size_t>(sg.b) * p.h + head0 + (row_ok ? r : 0)) * D;
+            if constexpr (REP == 1) {
+                if (have_o && live) {
+                    tc_fence_after();
+                    const bool row_ok = r < HS;
+                    const float inv = 1.f / l;
+                    __nv_bfloat16 *orow = p.out + (static_cast<size_t>(cur.b) * p.h + head0 + (row_ok ? r : 0)) * D;
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t raw[32];
+                        tmem_ld32(tO + cc * 32, raw);
+                        tmem_wait_ld();
+                        if (!row_ok) continue;
+                        if (whole) {
+                            uint32_t pk[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                pk[e] = pack_bf16x2(__uint_as_float(raw[2 * e]) * inv,
+                                                    __uint_as_float(raw[2 * e + 1]) * inv);
+                            uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        } else {
+                            uint4 *dst = reinterpret_cast<uint4 *>(slot + static_cast<size_t>(r) * D + cc * 32);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                dst[e] = make_uint4(raw[4 * e], raw[4 * e + 1], raw[4 * e + 2], raw[4 * e + 3]);
+                        }
+                    }
+                    if (!whole && row_ok) {
+                        slot[kSpRows * D + r] = m_used;
+                        slot[kSpRows * D + kSpRows + r] = l;
+                    }
+                }
+            } else {
+                // merge the copies of head hr through shared memory, 32 columns of O at a time;
+                // thread (kr, hr) then produces columns [kr CW, (kr + 1) CW) of each chunk.
+                // Every softmax thread takes the same barriers whatever happened above.
+                constexpr int CW = 32 / REP;
+                const bool go = bar_red_and(1, 128, have_o);
+                mrg_m[r] = m_used;
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                float M = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < REP; ++k) M = fmaxf(M, mrg_m[k * GP + hr]);
+                const float sc = m_used == -INFINITY ? 0.f : exp2f(m_used - M);
+                mrg_l[r] = l * sc;
+                const bool row_ok = go && hr < HS;
+                __nv_bfloat16 *orow = p.out + (static_cast<size_t>(cur.b) * p.h + head0 + (hr < HS ? hr : 0)) * D;
+                float inv = 0.f, lsum = 0.f;
+                if (go) tc_fence_after();
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t raw[32];
-                    tmem_ld32(tO + cc * 32, raw);
-                    tmem_wait_ld();
-                    if (!row_ok) continue;
-                    if (whole) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            pk[e] = pack_bf16x2(__uint_as_float(raw[2 * e]) * inv, __uint_as_float(raw[2 * e + 1]) * inv);
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    if (go) {
+                        tmem_ld32(tO + cc * 32, raw);
+                        tmem_wait_ld();
                     } else {
-                        uint4 *dst = reinterpret_cast<uint4 *>(slot + static_cast<size_t>(r) * D + cc * 32);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) dst[e] = make_uint4(raw[4 * e], raw[4 * e + 1], raw[4 * e + 2], raw[4 * e + 3]);
+                        for (int e = 0; e < 32; ++e) raw[e] = 0u;
                     }
+                    float4 *mine = reinterpret_cast<float4 *>(mrg + r * kSpMrgStride);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        mine[e] = make_float4(__uint_as_float(raw[4 * e]) * sc, __uint_as_float(raw[4 * e + 1]) * sc,
+                                              __uint_as_float(raw[4 * e + 2]) * sc,
+                                              __uint_as_float(raw[4 * e + 3]) * sc);
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    if (cc == 0) {
+#pragma unroll
+                        for (int k = 0; k < REP; ++k) lsum += mrg_l[k * GP + hr];
+                        inv = 1.f / lsum;
+                    }
+                    float acc[CW];
+#pragma unroll
+                    for (int e = 0; e < CW; ++e) acc[e] = 0.f;
+#pragma unroll
+                    for (int k = 0; k < REP; ++k) {
+                        const float4 *src = reinterpret_cast<const float4 *>(mrg + (k * GP + hr) * kSpMrgStride + kr * CW);
+#pragma unroll
+                        for (int e = 0; e < CW / 4; ++e) {
+                            const float4 v = src[e];
+                            acc[4 * e] += v.x;
+                            acc[4 * e + 1] += v.y;
+                            acc[4 * e + 2] += v.z;
+                            acc[4 * e + 3] += v.w;
+                        }
+                    }
+                    if (row_ok) {
+                        const int col = cc * 32 + kr * CW;
+                        if (whole) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
+#pragma unroll
+                            for (int e = 0; e < CW / 8; ++e)
+                                dst[e] = make_uint4(pack_bf16x2(acc[8 * e] * inv, acc[8 * e + 1] * inv),
+                                                    pack_bf16x2(acc[8 * e + 2] * inv, acc[8 * e + 3] * inv),
+                                                    pack_bf16x2(acc[8 * e + 4] * inv, acc[8 * e + 5] * inv),
+                                                    pack_bf16x2(acc[8 * e + 6] * inv, acc[8 * e + 7] * inv));
+                        } else {
+                            float4 *dst = reinterpret_cast<float4 *>(slot + static_cast<size_t>(hr) * D + col);
+#pragma unroll
+                            for (int e = 0; e < CW / 4; ++e)
+                                dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
+                        }
+                    }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");   // the buffer is free for the next chunk
                 }
-                if (!whole && row_ok) {
-                    slot[kSpRows * D + r] = m_used;
-                    slot[kSpRows * D + kSpRows + r] = l;
+                if (row_ok && !whole && kr == 0) {
+                    slot[kSpRows * D + hr] = M;
+                    slot[kSpRows * D + kSpRows + hr] = lsum;
                 }
             }
             tc_fence_before();
@@ -1240,12 +1432,12 @@ size_t split_workspace_bytes(int B, int h, int n_kv, int d) {
                     : split_workspace_bytes_t<64>(B, n_kv, slices, nctas);
 }
 
-template <int D>
+template <int D, int GP>
 static int launch_split_t(const void *q, const void *k, const void *v, long long cache_rows, const int32_t *seqlens,
                           void *out, int B, int h, int n_kv, float scale, void *workspace, size_t ws_bytes,
                           cudaStream_t stream) {
     using SG = SplitGeom<D>;
-    auto kern = gqa_decode_split_kernel<D>;
+    auto kern = gqa_decode_split_kernel<D, GP>;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 3;
     static std::atomic<unsigned long long> attr_done{0};
@@ -1255,20 +1447,13 @@ static int launch_split_t(const void *q, const void *k, const void *v, long long
         return 3;
     const int G = h / n_kv;
     const int slices = (G + kSpRows - 1) / kSpRows;
+    if (GP < kSpRows && G > GP) return 2;   // (the dispatcher never asks for this)
     const int nctas = gqa_host::sm_count();
     if (static_cast<long long>(n_kv) * slices * B > (1LL << 24)) return 2;   // segment indices stay int
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
         ws_bytes < split_workspace_bytes_t<D>(B, n_kv, slices, nctas))
         return 1;
-    CUtensorMap tq, tk, tv;
-    {
-        // q [B, h, D]: boxes of 64 dims x min(128, h) heads; rows past h read as zeros, rows of
-        // other groups are never stored
-        const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(h), static_cast<uint64_t>(B)};
-        const uint64_t strides[2] = {static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(h) * D * 2};
-        const uint32_t box[3] = {64, static_cast<uint32_t>(std::min(kSpRows, h)), 1};
-        if (!gqa_host::encode_tensor_map(&tq, q, 3, dims, strides, box)) return 3;
-    }
+    CUtensorMap tk, tv;
     {
         const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(n_kv),
                                   static_cast<uint64_t>(std::max(cache_rows, 1LL))};
@@ -1289,13 +1474,13 @@ static int launch_split_t(const void *q, const void *k, const void *v, long long
     prm.G = G;
     prm.slices = slices;
     prm.nctas = nctas;
-    prm.q_bytes = static_cast<uint32_t>(D * 2 * std::min(kSpRows, h));
+    prm.q_bytes = 0;   // (Q goes to TMEM through registers)
     prm.cache_rows = cache_rows;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.status = gqa_host::device_status();
     if (!prm.status) return 3;
     GQA_SET_TEST_STALL(prm);
-    kern<<<nctas, kSpThreads, SG::kTotal, stream>>>(tq, tk, tv, prm);
+    kern<<<nctas, kSpThreads, SG::kTotal, stream>>>(tk, tv, prm);
     if (cudaGetLastError() != cudaSuccess) return 3;
     gqa_decode_split_merge_kernel<D><<<dim3(static_cast<unsigned>(n_kv * slices * B), std::min(G, kSpRows)), 128, 0,
                                        stream>>>(prm.part, prm.seg, prm.out, B, h, G, slices, kSpRows);
@@ -1362,19 +1547,31 @@ static int launch_split_tok(const void *q, const void *k, const void *v, long lo
     return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }
 
+// Per group size, the faster kernel as measured: the tokens-as-rows kernel up to 32
+// heads (d = 128), the heads-as-rows kernel (with 2 copies of the group) up to 64,
+// and in slices of 128 heads above; at d = 64 the heads-as-rows kernel throughout.
 int launch_decode_split(const void *q, const void *k, const void *v, long long cache_rows, const int32_t *seqlens,
                         void *out, int B, int h, int n_kv, int d, float scale, void *workspace, size_t ws_bytes,
                         cudaStream_t stream) {
     const int G = h / n_kv;
-    if (d == 128 && G <= 16)
-        return launch_split_tok<16>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
-    if (d == 128 && G <= 32)
-        return launch_split_tok<32>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
-    if (d == 128 && G <= 64)
-        return launch_split_tok<64>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
-    if (d == 128)
-        return launch_split_t<128>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
-    return launch_split_t<64>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
+    if (d == 128) {
+        if (G <= 16)
+            return launch_split_tok<16>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes,
+                                        stream);
+        if (G <= 32)
+            return launch_split_tok<32>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes,
+                                        stream);
+        if (G <= 64)
+            return launch_split_t<128, 64>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes,
+                                           stream);
+        return launch_split_t<128, 128>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes,
+                                        stream);
+    }
+    if (G <= 32)
+        return launch_split_t<64, 32>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
+    if (G <= 64)
+        return launch_split_t<64, 64>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
+    return launch_split_t<64, 128>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------
