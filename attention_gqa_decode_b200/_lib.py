@@ -187,12 +187,15 @@ def prefill(q, k, v, causal: bool = True, scale: float | None = None, out=None, 
 
 
 # decode() sends a call to the split-KV kernels (gqa_decode_split) when the cache holds
-# at least SPLIT_MIN_MEAN_ROWS rows per sequence and either the groups are wide
-# (>= SPLIT_MIN_GROUP query heads per KV head) or there are too few (sequence, KV
-# head) units for the cluster kernel's at most 8 splits each to reach every SM;
-# everything else goes to the cluster kernel (gqa_decode_rows).  Measured on B200:
-# G = 128: split 1.6 TB/s, cluster 1.1; B4 h64 n_kv1 L32768: split 1.5 TB/s, cluster
-# 0.4; the GQA and MQA decode workloads: cluster 5.6 / 4.3, split 4.4 / 3.9.
+# at least SPLIT_MIN_MEAN_ROWS rows per sequence and either the groups are mid-sized at
+# d = 128 (SPLIT_WARP_GROUPS: the balanced warp-level kernel), wide (>= SPLIT_MIN_GROUP
+# query heads per KV head) or there are too few (sequence, KV head) units for the
+# cluster kernel's at most 8 splits each to reach every SM; everything else goes to the
+# cluster kernel (gqa_decode_rows).  Measured on B200 (graph replay, caches rotated past
+# L2): MQA B64 h32 L8192: split 4.60 TB/s, cluster 4.49; ragged B32 h64 n_kv1: split
+# 2.15, cluster 1.27; B4 h64 n_kv1 L32768: split 2.07, cluster 0.39; G = 128: split 1.6,
+# cluster 1.1; the GQA workload (G = 8): cluster 5.6, split 4.4.
+SPLIT_WARP_GROUPS = (17, 64)
 SPLIT_MIN_GROUP = 128
 SPLIT_MIN_MEAN_ROWS = 256
 _sm_counts = {}
@@ -214,6 +217,8 @@ def use_split(q, k_cache) -> bool:
     if n_kv <= 0 or h % n_kv or T < SPLIT_MIN_MEAN_ROWS * B:
         return False
     G = h // n_kv
+    if q.shape[2] == 128 and SPLIT_WARP_GROUPS[0] <= G <= SPLIT_WARP_GROUPS[1]:
+        return True
     units = B * n_kv * -(-G // 64)
     return G >= SPLIT_MIN_GROUP or units * 8 < _sm_count(q.device)
 

@@ -49,6 +49,7 @@
 // initialisation.
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -150,6 +151,82 @@ __device__ __forceinline__ int split_owner(long long w, long long W, int nc) {
     return static_cast<int>(((w + 1) * nc - 1) / W);
 }
 
+// T = the batch's tokens per (KV head, slice): the sum of the cut lengths (a
+// sequence is cut where its rows would pass the caches' rows, and reported;
+// offsets use the uncut lengths, as the packed layout does).  A sequence with
+// no tokens gets a zero output row for every head and a (-1, -1) segment
+// record, from CTA b % NC.  Called by all NT threads of the block; scan = 8
+// long longs of shared memory.
+template <int D, int NT>
+__device__ long long split_batch_tokens(const SplitParams &p, long long *scan, int c, int NC) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    long long T = 0, base_off = 0;
+    for (int b0 = 0; b0 < p.B; b0 += NT) {
+        const int bb = b0 + threadIdx.x;
+        const long long l = bb < p.B ? max(p.seqlens[bb], 0) : 0;
+        // block-wide exclusive scan of l (uncut offsets within this chunk)
+        long long x = l;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) scan[warp] = x;
+        __syncthreads();
+        long long before = 0, chunk = 0;
+        for (int w = 0; w < NT / 32; ++w) {
+            if (w < warp) before += scan[w];
+            chunk += scan[w];
+        }
+        const long long off_b = base_off + before + x - l;
+        const long long cut = bb < p.B ? max(0LL, min(l, p.cache_rows - off_b)) : 0;
+        if (cut < l) record_status(p.status, kStatusInvalid);
+        if (bb < p.B && cut == 0 && bb % NC == c) {   // no tokens: a zero output row for every head
+            uint4 *o4 = reinterpret_cast<uint4 *>(p.out + static_cast<size_t>(bb) * p.h * D);
+            for (int i = 0; i < p.h * D / 8; ++i) o4[i] = make_uint4(0u, 0u, 0u, 0u);
+            for (int gs = 0; gs < p.n_kv * p.slices; ++gs) p.seg[gs * p.B + bb] = make_int2(-1, -1);
+        }
+        // block-wide sum of the cut lengths
+        long long s = cut;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        __syncthreads();
+        if (lane == 0) scan[warp] = s;
+        __syncthreads();
+        for (int w = 0; w < NT / 32; ++w) T += scan[w];
+        base_off += chunk;
+        __syncthreads();
+    }
+    return T;
+}
+
+// A cursor over the work range [w_lo, w_hi): whole (KV head, slice) blocks,
+// then whole sequences, before w_lo are skipped
+__device__ SplitCursor split_cursor_at(const SplitParams &p, long long T, long long w_lo, long long w_hi) {
+    SplitCursor cu;
+    cu.p = &p;
+    cu.T = T;
+    cu.w_cur = w_lo;
+    cu.w_hi = w_hi;
+    cu.gs = 0;
+    cu.b = 0;
+    cu.off = 0;
+    cu.wb = 0;
+    if (T > 0) {
+        cu.gs = static_cast<int>(w_lo / T);
+        long long r = w_lo - cu.gs * T;
+        while (cu.b < p.B) {
+            const int L = cu.cut_len(cu.b, cu.off);
+            if (r < L) break;
+            r -= L;
+            cu.wb += L;
+            cu.off += max(p.seqlens[cu.b], 0);
+            ++cu.b;
+        }
+    }
+    return cu;
+}
+
 // bar.red.and over the first n threads of the block on named barrier id: true iff
 // pred holds in every one of them
 __device__ __forceinline__ bool bar_red_and(int id, int n, bool pred) {
@@ -228,49 +305,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         tmem_relinquish();
     }
 
-    // ---- the batch's tokens per (KV head, slice): T = sum of the cut lengths
-    // (a sequence is cut where its rows would pass the caches' rows; offsets use
-    // the uncut lengths, as the packed layout does)
-    long long T = 0;
-    {
-        long long base_off = 0;
-        for (int b0 = 0; b0 < p.B; b0 += kSpThreads) {
-            const int bb = b0 + threadIdx.x;
-            const long long l = bb < p.B ? max(p.seqlens[bb], 0) : 0;
-            // block-wide exclusive scan of l (uncut offsets within this chunk)
-            long long x = l;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const long long y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            if (lane == 31) scan[warp] = x;
-            __syncthreads();
-            long long before = 0, chunk = 0;
-            for (int w = 0; w < kSpThreads / 32; ++w) {
-                if (w < warp) before += scan[w];
-                chunk += scan[w];
-            }
-            const long long off_b = base_off + before + x - l;
-            const long long cut = bb < p.B ? max(0LL, min(l, p.cache_rows - off_b)) : 0;
-            if (cut < l) record_status(p.status, kStatusInvalid);
-            if (bb < p.B && cut == 0 && bb % NC == c) {   // no tokens: a zero output row for every head
-                uint4 *o4 = reinterpret_cast<uint4 *>(p.out + static_cast<size_t>(bb) * p.h * D);
-                for (int i = 0; i < p.h * D / 8; ++i) o4[i] = make_uint4(0u, 0u, 0u, 0u);
-                for (int gs = 0; gs < p.n_kv * p.slices; ++gs) p.seg[gs * p.B + bb] = make_int2(-1, -1);
-            }
-            // block-wide sum of the cut lengths
-            long long s = cut;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            __syncthreads();
-            if (lane == 0) scan[warp] = s;
-            __syncthreads();
-            for (int w = 0; w < kSpThreads / 32; ++w) T += scan[w];
-            base_off += chunk;
-            __syncthreads();
-        }
-    }
+    const long long T = split_batch_tokens<D, kSpThreads>(p, scan, c, NC);
     const long long W = static_cast<long long>(p.n_kv) * p.slices * T;
     // with fewer tokens than CTAs, only the first W CTAs take work (one token each), so
     // that every CTA between a segment's first and last owner holds a piece of it
@@ -283,31 +318,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    auto cursor = [&]() {
-        SplitCursor cu;
-        cu.p = &p;
-        cu.T = T;
-        cu.w_cur = w_lo;
-        cu.w_hi = w_hi;
-        cu.gs = 0;
-        cu.b = 0;
-        cu.off = 0;
-        cu.wb = 0;
-        // skip whole (KV head, slice) blocks, then whole sequences, before w_lo
-        if (T > 0) {
-            cu.gs = static_cast<int>(w_lo / T);
-            long long r = w_lo - cu.gs * T;
-            while (cu.b < p.B) {
-                const int L = cu.cut_len(cu.b, cu.off);
-                if (r < L) break;
-                r -= L;
-                cu.wb += L;
-                cu.off += max(p.seqlens[cu.b], 0);
-                ++cu.b;
-            }
-        }
-        return cu;
-    };
+    auto cursor = [&]() { return split_cursor_at(p, T, w_lo, w_hi); };
     auto n_stages = [](const SplitSeg &s) { return (s.t1 - s.t0 + kSpTok - 1) / kSpTok; };
 
     if (warp == 4) {
@@ -885,45 +896,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         reinterpret_cast<uint4 *>(sP)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
 
-    // ---- T = sum of the cut lengths; zero rows for sequences with no tokens (as the other kernel)
-    long long T = 0;
-    {
-        long long base_off = 0;
-        for (int b0 = 0; b0 < p.B; b0 += kSpThreads) {
-            const int bb = b0 + threadIdx.x;
-            const long long l = bb < p.B ? max(p.seqlens[bb], 0) : 0;
-            long long x = l;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const long long y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            if (lane == 31) scan[warp] = x;
-            __syncthreads();
-            long long before = 0, chunk = 0;
-            for (int w = 0; w < kSpThreads / 32; ++w) {
-                if (w < warp) before += scan[w];
-                chunk += scan[w];
-            }
-            const long long off_b = base_off + before + x - l;
-            const long long cut = bb < p.B ? max(0LL, min(l, p.cache_rows - off_b)) : 0;
-            if (cut < l) record_status(p.status, kStatusInvalid);
-            if (bb < p.B && cut == 0 && bb % NC == c) {
-                uint4 *o4 = reinterpret_cast<uint4 *>(p.out + static_cast<size_t>(bb) * p.h * D);
-                for (int i = 0; i < p.h * D / 8; ++i) o4[i] = make_uint4(0u, 0u, 0u, 0u);
-                for (int gs = 0; gs < p.n_kv * p.slices; ++gs) p.seg[gs * p.B + bb] = make_int2(-1, -1);
-            }
-            long long s = cut;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            __syncthreads();
-            if (lane == 0) scan[warp] = s;
-            __syncthreads();
-            for (int w = 0; w < kSpThreads / 32; ++w) T += scan[w];
-            base_off += chunk;
-            __syncthreads();
-        }
-    }
+    const long long T = split_batch_tokens<D, kSpThreads>(p, scan, c, NC);
     const long long W = static_cast<long long>(p.n_kv) * p.slices * T;
     const int NCe = W < NC ? static_cast<int>(W) : NC;
     const long long w_lo = c < NCe ? W * c / NCe : W, w_hi = c < NCe ? W * (c + 1) / NCe : W;
@@ -934,30 +907,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    auto cursor = [&]() {
-        SplitCursor cu;
-        cu.p = &p;
-        cu.T = T;
-        cu.w_cur = w_lo;
-        cu.w_hi = w_hi;
-        cu.gs = 0;
-        cu.b = 0;
-        cu.off = 0;
-        cu.wb = 0;
-        if (T > 0) {
-            cu.gs = static_cast<int>(w_lo / T);
-            long long r = w_lo - cu.gs * T;
-            while (cu.b < p.B) {
-                const int L = cu.cut_len(cu.b, cu.off);
-                if (r < L) break;
-                r -= L;
-                cu.wb += L;
-                cu.off += max(p.seqlens[cu.b], 0);
-                ++cu.b;
-            }
-        }
-        return cu;
-    };
+    auto cursor = [&]() { return split_cursor_at(p, T, w_lo, w_hi); };
     auto n_stages = [](const SplitSeg &sg) { return (sg.t1 - sg.t0 + kTkTok - 1) / kTkTok; };
 
     if (warp == 4) {
@@ -1350,16 +1300,420 @@ __global__ void __launch_bounds__(kSpThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Warp-level MMAs over the balanced partition, for groups of 17 to 64 heads
+// (d = 128).  At these group sizes the rows of a 128-row tcgen05 MMA are
+// mostly padding (or copies), while mma.sync m16n8k16 fits the group: the
+// consumer warps are those of the cluster decode kernel -- warp (mi, ti) takes
+// query heads [16 mi, 16 mi + 16) as the M rows and tokens [ti TOK / WT,
+// (ti + 1) TOK / WT) of every stage, S = Q K^T and O += P V with K and V read
+// from the TMA-filled ring by ldmatrix, the online softmax on the fragments --
+// but the work is the batch's tokens divided evenly among two CTAs per SM, as
+// in the kernels above, instead of a fixed number of splits per sequence.  A
+// segment's two token groups (WT = 2) merge through a small shared buffer; a
+// segment cut between CTAs leaves a partial result (a slot of 64 rows) for
+// the merge kernel.
+constexpr int kBlTok = 64;             // tokens per stage
+constexpr int kBlStages = 3;           // ring depth (two CTAs per SM)
+constexpr int kBlWarps = 4;            // consumer warps
+constexpr int kBlThreads = (kBlWarps + 1) * 32;
+constexpr int kBlRows = 64;            // heads of a partial slot
+constexpr int kBlCtasPerSm = 2;
+
+struct BalGeom {   // d = 128, bf16
+    static constexpr int D = 128;
+    static constexpr uint32_t kPanelBytes = kBlTok * 128;          // 64 tokens x 64 dims
+    static constexpr uint32_t kTileBytes = (D / 64) * kPanelBytes;  // K or V of a stage
+    static constexpr uint32_t kStageBytes = 2 * kTileBytes;
+    static constexpr uint32_t kRing = kBlStages * kStageBytes;
+    static constexpr uint32_t kMrg = (2 * 16 * 64 + 2 * 2 * 16) * 4;   // 2 m-tiles: half of O (16 x 64), m, l
+    static constexpr uint32_t kCtrl = 256;
+    static constexpr uint32_t kTotal = kRing + kMrg + kCtrl + 1024;
+    static constexpr uint32_t kPartFloats = kBlRows * D + 2 * kBlRows;
+};
+
+template <int WT>
+__global__ void __launch_bounds__(kBlThreads, kBlCtasPerSm)
+    gqa_decode_bal_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                          const SplitParams p) {
+    using BG = BalGeom;
+    constexpr int D = BG::D;
+    constexpr int TOK = kBlTok;
+    constexpr int RB = 128;                  // bytes of a token row in a panel
+    constexpr int KSTEPS = D / 16;
+    constexpr int NT_O = D / 8;
+    constexpr int TWARP = TOK / WT;          // tokens of a stage one warp handles
+    constexpr int TPW = TWARP < 32 ? TWARP : 32;   // tokens per pass (O takes 64 registers)
+    constexpr int NPASS = TWARP / TPW;
+    constexpr int NTS = TPW / 8;             // n-tiles of the scores of a pass
+    constexpr int KKS = TPW / 16;            // k-steps of its P V
+    static_assert(WT == 1 || WT == 2, "one or two token groups");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *mrg = reinterpret_cast<float *>(smem + BG::kRing);    // [2][16][64]: token group 1's O, one half
+    float *mrg_ml = mrg + 2 * 16 * 64;                          // [2][2][16]: its m and l
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + BG::kRing + BG::kMrg);
+    uint64_t *empty = full + kBlStages;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kBlStages);
+    long long *scan = reinterpret_cast<long long *>(empty + kBlStages + 1);   // [8]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x, NC = p.nctas;
+    const int HS = p.G;                      // <= 64: one slice
+    const int WM = (HS + 15) >> 4;           // m-tiles (WM * WT <= 4, chosen by the host)
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kBlStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], WM * WT);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == kBlWarps && lane == 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    const long long T = split_batch_tokens<D, kBlThreads>(p, scan, c, NC);
+    __syncthreads();   // (the barriers' initialisation is visible to every thread)
+    const long long W = static_cast<long long>(p.n_kv) * T;
+    const int NCe = W < NC ? static_cast<int>(W) : NC;
+    const long long w_lo = c < NCe ? W * c / NCe : W, w_hi = c < NCe ? W * (c + 1) / NCe : W;
+    auto n_stages = [](const SplitSeg &s) { return (s.t1 - s.t0 + TOK - 1) / TOK; };
+
+    if (warp == kBlWarps) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            SplitCursor cu = split_cursor_at(p, T, w_lo, w_hi);
+            SplitSeg sg;
+            int gi = 0;
+            const int first_loaded = GQA_STALLED(p) ? 1 : 0;   // wait-test build: stage 0 never arrives
+            bool ok = true;
+            while (ok && cu.next(sg)) {
+                const int g = sg.gs;
+                const int n = n_stages(sg);
+                for (int i = 0; i < n; ++i, ++gi) {
+                    const int slot = gi % kBlStages, use = gi / kBlStages;
+                    if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    if (gi < first_loaded) continue;
+                    // the stage's box may run past the segment (into rows the consumers mask)
+                    const int z = static_cast<int>(sg.off) + sg.t0 + i * TOK;
+                    uint8_t *kd = smem + slot * BG::kStageBytes;
+                    mbar_arrive_expect_tx(&full[slot], BG::kStageBytes);
+#pragma unroll
+                    for (int pp = 0; pp < D / 64; ++pp) {
+                        tma_load_3d(kd + pp * BG::kPanelBytes, &tm_k, &full[slot], pp * 64, g, z);
+                        tma_load_3d(kd + BG::kTileBytes + pp * BG::kPanelBytes, &tm_v, &full[slot], pp * 64, g, z);
+                    }
+                }
+            }
+            if (*abort_flag) {   // let the copies in flight land before the CTA exits
+                for (int i = max(first_loaded, gi - kBlStages); i < gi; ++i)
+                    mbar_wait_drain(&full[i % kBlStages], (i / kBlStages) & 1, p.status);
+            }
+        }
+        __syncwarp();
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const int mi = warp / WT, ti = warp % WT;
+    const bool consumer = mi < WM;
+    if (WT == 1 && !consumer) return;        // (WT = 2 runs with WM = 2: every warp consumes)
+    const float cl2 = p.scale_log2;
+    const int r0 = mi * 16 + (lane >> 2), r1 = r0 + 8;   // this lane's heads (rows of the m-tile)
+    const int cq = 2 * (lane & 3);
+    // ldmatrix lane roles
+    const uint32_t lrow = ((lane >> 4) & 1) * 8 + (lane & 7);   // QK: token within a 16-token pair
+    const uint32_t lchk = (lane >> 3) & 1;                      // QK: low/high 8 dims of a k-step
+    const uint32_t frow = ((lane >> 3) & 1) * 8 + (lane & 7);   // PV: token within 16 tokens
+    const uint32_t fchk = lane >> 4;                            // PV: chunk within a pair of chunks
+
+    SplitCursor cu = split_cursor_at(p, T, w_lo, w_hi);
+    SplitSeg sg;
+    int gi0 = 0;
+    bool ok = true;
+    while (cu.next(sg)) {
+        const int g = sg.gs;
+        const int head0 = g * p.G;
+        const int n = n_stages(sg);
+        const bool split = sg.L <= kSpSplitAllBelow;   // short sequence: the weights' bf16 remainders too
+        float o[NT_O][4];
+        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+#pragma unroll
+        for (int nt = 0; nt < NT_O; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+        if (consumer && ok) {
+            // Q fragments of m-tile mi (rows = the group's heads)
+            const __nv_bfloat16 *qb = p.q + (static_cast<size_t>(sg.b) * p.h + head0) * D;
+            uint32_t qa[KSTEPS][4];
+#pragma unroll
+            for (int ks = 0; ks < KSTEPS; ++ks) {
+                const int cc = ks * 16 + cq;
+                qa[ks][0] = r0 < HS ? *reinterpret_cast<const uint32_t *>(qb + r0 * D + cc) : 0u;
+                qa[ks][1] = r1 < HS ? *reinterpret_cast<const uint32_t *>(qb + r1 * D + cc) : 0u;
+                qa[ks][2] = r0 < HS ? *reinterpret_cast<const uint32_t *>(qb + r0 * D + cc + 8) : 0u;
+                qa[ks][3] = r1 < HS ? *reinterpret_cast<const uint32_t *>(qb + r1 * D + cc + 8) : 0u;
+            }
+            // the stage loop, compiled with and without the remainder products (registers)
+            auto stages = [&](auto split_tag) {
+                constexpr bool SPLIT = decltype(split_tag)::value;
+                for (int i = 0; i < n; ++i) {
+                    const int gi = gi0 + i;
+                    const int slot = gi % kBlStages, use = gi / kBlStages;
+                    const bool landed = mbar_wait(&full[slot], use & 1, abort_flag, p.status);
+                    if (!__all_sync(0xffffffffu, landed)) {   // warp-uniform: the mma/ldmatrix below are .aligned
+                        ok = false;
+                        break;
+                    }
+                    // valid rows of the stage: [0, row_hi); the rest belong to other CTAs or sequences
+                    const int row_hi = min(TOK, sg.t1 - (sg.t0 + i * TOK));
+                    const uint32_t stage = smem_u32(smem + slot * BG::kStageBytes);
+    #pragma unroll
+                    for (int pass = 0; pass < NPASS; ++pass) {
+                        const int tw0 = ti * TWARP + pass * TPW;   // first row of this pass
+                        if (row_hi <= tw0) continue;                // no valid row here
+                        const bool partial = row_hi < tw0 + TPW;
+                        const uint32_t kbase = stage + tw0 * RB;
+                        const uint32_t vbase = kbase + BG::kTileBytes;
+
+                        // S = Q K^T  (16 heads x TPW tokens)
+                        float s[NTS][4];
+    #pragma unroll
+                        for (int nt = 0; nt < NTS; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+    #pragma unroll
+                        for (int ks = 0; ks < KSTEPS; ++ks) {
+                            const uint32_t chunk = 2 * ks + lchk;
+                            const uint32_t hbase = kbase + (chunk >> 3) * BG::kPanelBytes + (((chunk & 7) ^ (lane & 7)) << 4);
+    #pragma unroll
+                            for (int np = 0; np < NTS / 2; ++np) {
+                                uint32_t b0, b1, b2, b3;
+                                ldmatrix_x4(b0, b1, b2, b3, hbase + (np * 16 + lrow) * RB);
+                                mma_bf16_16816(s[2 * np], qa[ks], b0, b1);
+                                mma_bf16_16816(s[2 * np + 1], qa[ks], b2, b3);
+                            }
+                        }
+                        if (partial) {
+    #pragma unroll
+                            for (int nt = 0; nt < NTS; ++nt)
+    #pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    if (tw0 + nt * 8 + cq + (e & 1) >= row_hi) s[nt][e] = -INFINITY;
+                        }
+                        // online softmax over these tokens (rows r0 and r1 of the m-tile)
+                        float mx[2] = {-INFINITY, -INFINITY};
+    #pragma unroll
+                        for (int nt = 0; nt < NTS; ++nt) {
+                            mx[0] = fmax3(mx[0], s[nt][0], s[nt][1]);
+                            mx[1] = fmax3(mx[1], s[nt][2], s[nt][3]);
+                        }
+                        float alpha[2];
+    #pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+                            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+                            const float m_new = fmaxf(m_run[r], mx[r] * cl2);   // mx is finite: >= 1 valid token
+                            alpha[r] = exp2f(m_run[r] - m_new);
+                            m_run[r] = m_new;
+                            l_run[r] *= alpha[r];
+                        }
+    #pragma unroll
+                        for (int nt = 0; nt < NT_O; ++nt) {
+                            o[nt][0] *= alpha[0];
+                            o[nt][1] *= alpha[0];
+                            o[nt][2] *= alpha[1];
+                            o[nt][3] *= alpha[1];
+                        }
+                        // P as bf16 A fragments; the running sums add the rounded weights
+                        uint32_t pa[KKS][4], par[KKS][4];   // the weights and, for short sequences, their remainders
+                        float2 ls0 = make_float2(0.f, 0.f), ls1 = make_float2(0.f, 0.f);
+    #pragma unroll
+                        for (int nt = 0; nt < NTS; ++nt) {
+                            const float2 y0 = ffma2_bcast(s[nt][0], s[nt][1], cl2, -m_run[0]);
+                            const float2 y1 = ffma2_bcast(s[nt][2], s[nt][3], cl2, -m_run[1]);
+                            float e0 = exp2f(y0.x), e1 = exp2f(y0.y), e2 = exp2f(y1.x), e3 = exp2f(y1.y);
+                            if (partial) {   // masked tokens add nothing (also when the scale is 0)
+                                const int row = tw0 + nt * 8 + cq;
+                                if (row >= row_hi) e0 = e2 = 0.f;
+                                if (row + 1 >= row_hi) e1 = e3 = 0.f;
+                            }
+                            const uint32_t lo = pack_bf16x2(e0, e1), hi = pack_bf16x2(e2, e3);
+                            const float2 ul = unpack_bf16x2(lo), uh = unpack_bf16x2(hi);
+                            ls0 = fadd2(ls0, ul);
+                            ls1 = fadd2(ls1, uh);
+                            if constexpr (SPLIT) {   // remainders (exact in fp32), rounded to bf16 for a second product
+                                const uint32_t rl = pack_bf16x2(e0 - ul.x, e1 - ul.y);
+                                const uint32_t rh = pack_bf16x2(e2 - uh.x, e3 - uh.y);
+                                ls0 = fadd2(ls0, unpack_bf16x2(rl));
+                                ls1 = fadd2(ls1, unpack_bf16x2(rh));
+                                par[nt >> 1][(nt & 1) * 2 + 0] = rl;
+                                par[nt >> 1][(nt & 1) * 2 + 1] = rh;
+                            }
+                            pa[nt >> 1][(nt & 1) * 2 + 0] = lo;
+                            pa[nt >> 1][(nt & 1) * 2 + 1] = hi;
+                        }
+                        l_run[0] += ls0.x + ls0.y;
+                        l_run[1] += ls1.x + ls1.y;
+                        // O += P V.  On a partial pass the V values of invalid rows are zeroed in
+                        // registers (each half of a transposed fragment register is one token), so
+                        // that 0 * (whatever those rows hold) adds nothing.
+                        auto pv = [&](auto masked) {
+                            constexpr bool MASKED = decltype(masked)::value;
+    #pragma unroll
+                            for (int kk = 0; kk < KKS; ++kk) {
+                                uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
+                                if constexpr (MASKED) {
+                                    const int row = tw0 + kk * 16 + cq;   // this lane's tokens: row, row + 1 (and + 8)
+                                    mlo = (row < row_hi ? 0x0000FFFFu : 0u) | (row + 1 < row_hi ? 0xFFFF0000u : 0u);
+                                    mhi = (row + 8 < row_hi ? 0x0000FFFFu : 0u) | (row + 9 < row_hi ? 0xFFFF0000u : 0u);
+                                }
+                                const uint32_t rowaddr = vbase + (kk * 16 + frow) * RB;
+    #pragma unroll
+                                for (int dp = 0; dp < NT_O / 2; ++dp) {
+                                    const uint32_t chunk = 2 * dp + fchk;
+                                    uint32_t b0, b1, b2, b3;
+                                    ldmatrix_x4_trans(b0, b1, b2, b3,
+                                                      rowaddr + (chunk >> 3) * BG::kPanelBytes +
+                                                          (((chunk & 7) ^ (lane & 7)) << 4));
+                                    if constexpr (MASKED) {
+                                        b0 &= mlo;
+                                        b1 &= mhi;
+                                        b2 &= mlo;
+                                        b3 &= mhi;
+                                    }
+                                    mma_bf16_16816(o[2 * dp], pa[kk], b0, b1);
+                                    mma_bf16_16816(o[2 * dp + 1], pa[kk], b2, b3);
+                                    if constexpr (SPLIT) {
+                                        mma_bf16_16816(o[2 * dp], par[kk], b0, b1);
+                                        mma_bf16_16816(o[2 * dp + 1], par[kk], b2, b3);
+                                    }
+                                }
+                            }
+                        };
+                        if (partial)
+                            pv(std::true_type{});
+                        else
+                            pv(std::false_type{});
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[slot]);
+                }
+            };
+            if (split)
+                stages(std::true_type{});
+            else
+                stages(std::false_type{});
+        }
+        gi0 += n;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
+            l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
+        }
+
+        // ---- the segment's result: token group 1 hands its partial to group 0 through
+        // shared memory (half of O at a time), which merges and writes
+        if constexpr (WT == 2) {
+            const int lr0 = lane >> 2, lr1 = lr0 + 8;   // rows within the m-tile
+            float a_me[2] = {1.f, 1.f}, a_ot[2] = {0.f, 0.f};
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                if (ti == 1) {
+#pragma unroll
+                    for (int nt = 0; nt < NT_O / 2; ++nt) {
+                        const int col = nt * 8 + cq;
+                        float *m0 = mrg + (mi * 16 + lr0) * 64 + col, *m1 = mrg + (mi * 16 + lr1) * 64 + col;
+                        *reinterpret_cast<float2 *>(m0) = make_float2(o[half * 8 + nt][0], o[half * 8 + nt][1]);
+                        *reinterpret_cast<float2 *>(m1) = make_float2(o[half * 8 + nt][2], o[half * 8 + nt][3]);
+                    }
+                    if (half == 0 && (lane & 3) == 0) {
+                        mrg_ml[(mi * 2 + 0) * 16 + lr0] = m_run[0];
+                        mrg_ml[(mi * 2 + 0) * 16 + lr1] = m_run[1];
+                        mrg_ml[(mi * 2 + 1) * 16 + lr0] = l_run[0];
+                        mrg_ml[(mi * 2 + 1) * 16 + lr1] = l_run[1];
+                    }
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (ti == 0) {
+                    if (half == 0) {
+#pragma unroll
+                        for (int r = 0; r < 2; ++r) {
+                            const int lr = r ? lr1 : lr0;
+                            const float mo = mrg_ml[(mi * 2 + 0) * 16 + lr], lo = mrg_ml[(mi * 2 + 1) * 16 + lr];
+                            const float M = fmaxf(m_run[r], mo);
+                            a_me[r] = M == -INFINITY ? 0.f : exp2f(m_run[r] - M);
+                            a_ot[r] = M == -INFINITY ? 0.f : exp2f(mo - M);
+                            l_run[r] = l_run[r] * a_me[r] + lo * a_ot[r];
+                            m_run[r] = M;
+                        }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT_O / 2; ++nt) {
+                        const int col = nt * 8 + cq;
+                        const float2 x0 = *reinterpret_cast<const float2 *>(mrg + (mi * 16 + lr0) * 64 + col);
+                        const float2 x1 = *reinterpret_cast<const float2 *>(mrg + (mi * 16 + lr1) * 64 + col);
+                        float *oo = o[half * 8 + nt];
+                        oo[0] = oo[0] * a_me[0] + x0.x * a_ot[0];
+                        oo[1] = oo[1] * a_me[0] + x0.y * a_ot[0];
+                        oo[2] = oo[2] * a_me[1] + x1.x * a_ot[1];
+                        oo[3] = oo[3] * a_me[1] + x1.y * a_ot[1];
+                    }
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");   // the buffer is free again
+            }
+        }
+        const int first_c = split_owner(sg.w, W, NCe), last_c = split_owner(sg.w + sg.L - 1, W, NCe);
+        const int sidx = g * p.B + sg.b;
+        if (ti == 0 && consumer && ok) {
+            if (first_c == last_c) {   // the whole sequence: O / l
+                __nv_bfloat16 *ob = p.out + (static_cast<size_t>(sg.b) * p.h + head0) * D;
+                const float inv0 = 1.f / l_run[0], inv1 = 1.f / l_run[1];
+#pragma unroll
+                for (int nt = 0; nt < NT_O; ++nt) {
+                    if (r0 < HS)
+                        *reinterpret_cast<uint32_t *>(ob + r0 * D + nt * 8 + cq) =
+                            pack_bf16x2(o[nt][0] * inv0, o[nt][1] * inv0);
+                    if (r1 < HS)
+                        *reinterpret_cast<uint32_t *>(ob + r1 * D + nt * 8 + cq) =
+                            pack_bf16x2(o[nt][2] * inv1, o[nt][3] * inv1);
+                }
+            } else {                   // a piece: unnormalised O, m, l into slot c + sidx
+                float *slot = p.part + static_cast<size_t>(c + sidx) * BG::kPartFloats;
+#pragma unroll
+                for (int nt = 0; nt < NT_O; ++nt) {
+                    if (r0 < HS) *reinterpret_cast<float2 *>(slot + r0 * D + nt * 8 + cq) = make_float2(o[nt][0], o[nt][1]);
+                    if (r1 < HS) *reinterpret_cast<float2 *>(slot + r1 * D + nt * 8 + cq) = make_float2(o[nt][2], o[nt][3]);
+                }
+                if ((lane & 3) == 0) {
+                    if (r0 < HS) {
+                        slot[kBlRows * D + r0] = m_run[0];
+                        slot[kBlRows * D + kBlRows + r0] = l_run[0];
+                    }
+                    if (r1 < HS) {
+                        slot[kBlRows * D + r1] = m_run[1];
+                        slot[kBlRows * D + kBlRows + r1] = l_run[1];
+                    }
+                }
+            }
+        }
+        // the segment's record for the merge kernel, from the CTA of its first piece
+        if (c == first_c && threadIdx.x == 0) p.seg[sidx] = make_int2(first_c, last_c);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // The merge of the pieces of the segments that were cut between CTAs, in a
 // second launch so that it runs on every SM at once: one block per (segment,
 // head), four warps each folding a quarter of the pieces with the log-sum-exp
 // rule (running max M, sum L, unnormalised O), then warp 0 folds the four.
 
-template <int D>
+template <int D, int ROWS>   // ROWS: heads of a partial slot (O [ROWS][D], then m [ROWS], l [ROWS])
 __global__ void __launch_bounds__(128)
     gqa_decode_split_merge_kernel(const float *part, const int2 *seg, __nv_bfloat16 *out, int B, int h, int G,
                                   int slices, int rows) {
-    constexpr uint32_t SLOT = SplitGeom<D>::kPartFloats;
+    constexpr uint32_t SLOT = ROWS * D + 2 * ROWS;
     __shared__ float sM[4], sL[4];
     __shared__ float4 sO[4][D / 4];
     const int sidx = blockIdx.x, hh = blockIdx.y;
@@ -1375,8 +1729,8 @@ __global__ void __launch_bounds__(128)
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int cc = info.x + warp; cc <= info.y; cc += 4) {
         const float *sp = part + static_cast<size_t>(cc + sidx) * SLOT;
-        const float m = __ldcg(sp + kSpRows * D + hh);
-        const float l = __ldcg(sp + kSpRows * D + kSpRows + hh);
+        const float m = __ldcg(sp + ROWS * D + hh);
+        const float l = __ldcg(sp + ROWS * D + ROWS + hh);
         const float4 o = act ? __ldcg(reinterpret_cast<const float4 *>(sp + static_cast<size_t>(hh) * D) + lane)
                              : make_float4(0.f, 0.f, 0.f, 0.f);
         const float M2 = fmaxf(M, m);
@@ -1410,6 +1764,15 @@ __global__ void __launch_bounds__(128)
 // ---------------------------------------------------------------------------
 // host side
 
+// The merge launch: one block per (segment, head)
+template <int D, int ROWS>
+static int launch_merge(const SplitParams &prm, int n_segments, int heads, cudaStream_t stream) {
+    gqa_decode_split_merge_kernel<D, ROWS><<<dim3(static_cast<unsigned>(n_segments), static_cast<unsigned>(heads)), 128,
+                                             0, stream>>>(prm.part, prm.seg, prm.out, prm.B, prm.h, prm.G, prm.slices,
+                                                          ROWS);
+    return cudaGetLastError() == cudaSuccess ? 0 : 3;
+}
+
 // bytes of the per-segment records at the start of the workspace (a multiple of 256)
 static size_t seg_bytes_for(int B, int n_kv, int slices) {
     const size_t ns = static_cast<size_t>(n_kv) * slices * B;
@@ -1424,12 +1787,29 @@ static size_t split_workspace_bytes_t(int B, int n_kv, int slices, int nctas) {
 }
 
 
+// The kernel gqa_decode_split runs for a shape (by group size, as measured): warp-level
+// MMAs over the balanced partition for 17 to 64 heads at d = 128, tokens as rows up to
+// 16, heads as rows otherwise.
+enum class SplitPath { kTok, kHeads, kBal };
+static SplitPath split_path(int h, int n_kv, int d) {
+    const int G = h / n_kv;
+    if (d == 128 && G > 16 && G <= kBlRows) return SplitPath::kBal;
+    if (d == 128 && G <= 16) return SplitPath::kTok;
+    return SplitPath::kHeads;
+}
+
+static size_t bal_workspace_bytes(int B, int n_kv, int nctas) {
+    return seg_bytes_for(B, n_kv, 1) +
+           (static_cast<size_t>(nctas) + static_cast<size_t>(n_kv) * B) * BalGeom::kPartFloats * sizeof(float);
+}
+
 size_t split_workspace_bytes(int B, int h, int n_kv, int d) {
     const int G = h / n_kv;
     const int slices = (G + kSpRows - 1) / kSpRows;
-    const int nctas = gqa_host::sm_count();
-    return d == 128 ? split_workspace_bytes_t<128>(B, n_kv, slices, nctas)
-                    : split_workspace_bytes_t<64>(B, n_kv, slices, nctas);
+    const int sms = gqa_host::sm_count();
+    if (split_path(h, n_kv, d) == SplitPath::kBal) return bal_workspace_bytes(B, n_kv, kBlCtasPerSm * sms);
+    return d == 128 ? split_workspace_bytes_t<128>(B, n_kv, slices, sms)
+                    : split_workspace_bytes_t<64>(B, n_kv, slices, sms);
 }
 
 template <int D, int GP>
@@ -1482,9 +1862,7 @@ static int launch_split_t(const void *q, const void *k, const void *v, long long
     GQA_SET_TEST_STALL(prm);
     kern<<<nctas, kSpThreads, SG::kTotal, stream>>>(tk, tv, prm);
     if (cudaGetLastError() != cudaSuccess) return 3;
-    gqa_decode_split_merge_kernel<D><<<dim3(static_cast<unsigned>(n_kv * slices * B), std::min(G, kSpRows)), 128, 0,
-                                       stream>>>(prm.part, prm.seg, prm.out, B, h, G, slices, kSpRows);
-    return cudaGetLastError() == cudaSuccess ? 0 : 3;
+    return launch_merge<D, kSpRows>(prm, n_kv * slices * B, std::min(G, kSpRows), stream);
 }
 
 // The tokens-as-rows kernel (d = 128, groups of at most 64 heads); the workspace
@@ -1542,31 +1920,77 @@ static int launch_split_tok(const void *q, const void *k, const void *v, long lo
     GQA_SET_TEST_STALL(prm);
     kern<<<nctas, kSpThreads, TG::kTotal, stream>>>(tq, tk, tv, prm);
     if (cudaGetLastError() != cudaSuccess) return 3;
-    gqa_decode_split_merge_kernel<128><<<dim3(static_cast<unsigned>(n_kv * B), G), 128, 0, stream>>>(
-        prm.part, prm.seg, prm.out, B, h, G, 1, kTkN);
-    return cudaGetLastError() == cudaSuccess ? 0 : 3;
+    return launch_merge<128, kSpRows>(prm, n_kv * B, G, stream);
 }
 
-// Per group size, the faster kernel as measured: the tokens-as-rows kernel up to 32
-// heads (d = 128), the heads-as-rows kernel (with 2 copies of the group) up to 64,
-// and in slices of 128 heads above; at d = 64 the heads-as-rows kernel throughout.
+template <int WT>
+static int launch_split_bal(const void *q, const void *k, const void *v, long long cache_rows, const int32_t *seqlens,
+                            void *out, int B, int h, int n_kv, float scale, void *workspace, size_t ws_bytes,
+                            cudaStream_t stream) {
+    using BG = BalGeom;
+    auto kern = gqa_decode_bal_kernel<WT>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 3;
+    static std::atomic<unsigned long long> attr_done{0};
+    if (!gqa_host::once_per_device(attr_done, dev, [&] {
+            return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BG::kTotal) == cudaSuccess;
+        }))
+        return 3;
+    const int G = h / n_kv;
+    const int WM = (G + 15) / 16;
+    if (G > kBlRows || WM * WT > kBlWarps || (WT == 2 && WM != 2)) return 2;   // (the dispatcher never asks)
+    const int nctas = kBlCtasPerSm * gqa_host::sm_count();
+    if (static_cast<long long>(n_kv) * B > (1LL << 24)) return 2;   // segment indices stay int
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || ws_bytes < bal_workspace_bytes(B, n_kv, nctas))
+        return 1;
+    CUtensorMap tk, tv;
+    {
+        const uint64_t dims[3] = {static_cast<uint64_t>(BG::D), static_cast<uint64_t>(n_kv),
+                                  static_cast<uint64_t>(std::max(cache_rows, 1LL))};
+        const uint64_t strides[2] = {static_cast<uint64_t>(BG::D) * 2, static_cast<uint64_t>(n_kv) * BG::D * 2};
+        const uint32_t box[3] = {64, 1, static_cast<uint32_t>(kBlTok)};
+        if (!gqa_host::encode_tensor_map(&tk, k, 3, dims, strides, box)) return 3;
+        if (!gqa_host::encode_tensor_map(&tv, v, 3, dims, strides, box)) return 3;
+    }
+    SplitParams prm = {};
+    prm.q = static_cast<const __nv_bfloat16 *>(q);
+    prm.seqlens = seqlens;
+    prm.out = static_cast<__nv_bfloat16 *>(out);
+    prm.seg = static_cast<int2 *>(workspace);
+    prm.part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + seg_bytes_for(B, n_kv, 1));
+    prm.B = B;
+    prm.h = h;
+    prm.n_kv = n_kv;
+    prm.G = G;
+    prm.slices = 1;
+    prm.nctas = nctas;
+    prm.q_bytes = 0;
+    prm.cache_rows = cache_rows;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.status = gqa_host::device_status();
+    if (!prm.status) return 3;
+    GQA_SET_TEST_STALL(prm);
+    kern<<<nctas, kBlThreads, BG::kTotal, stream>>>(tk, tv, prm);
+    if (cudaGetLastError() != cudaSuccess) return 3;
+    return launch_merge<BG::D, kBlRows>(prm, n_kv * B, G, stream);
+}
+
 int launch_decode_split(const void *q, const void *k, const void *v, long long cache_rows, const int32_t *seqlens,
                         void *out, int B, int h, int n_kv, int d, float scale, void *workspace, size_t ws_bytes,
                         cudaStream_t stream) {
     const int G = h / n_kv;
-    if (d == 128) {
-        if (G <= 16)
-            return launch_split_tok<16>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes,
-                                        stream);
+    const SplitPath path = split_path(h, n_kv, d);
+    if (path == SplitPath::kBal) {
         if (G <= 32)
-            return launch_split_tok<32>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes,
-                                        stream);
-        if (G <= 64)
-            return launch_split_t<128, 64>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes,
-                                           stream);
+            return launch_split_bal<2>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes,
+                                       stream);
+        return launch_split_bal<1>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
+    }
+    if (path == SplitPath::kTok)
+        return launch_split_tok<16>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
+    if (d == 128)
         return launch_split_t<128, 128>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes,
                                         stream);
-    }
     if (G <= 32)
         return launch_split_t<64, 32>(q, k, v, cache_rows, seqlens, out, B, h, n_kv, scale, workspace, ws_bytes, stream);
     if (G <= 64)

@@ -121,17 +121,22 @@ int gqa_decode_rows(const void *q, const void *k_cache, const void *v_cache, int
                     int B, int h, int n_kv, int d_h, float scale, cudaStream_t stream);
 
 /*
- * Decode with the batch's cached tokens divided evenly among the SMs, on the
- * 5th-generation tensor cores: the same result as gqa_decode_rows (same
- * arguments, same row check, same device status), built for groups of many
- * query heads per KV head (MQA, wide GQA) and for ragged lengths.  The query
- * heads of a group are the rows of the tensor-core products ("Multi-query
- * attention" (pranaymahendrakar), "Why this is a bandwidth argument, not a
- * FLOP argument": at h / n_kv query heads per KV head the step does h / n_kv
- * multiply-adds per cached element, too many for the warp-level path once
- * the group is wide), and a sequence whose tokens fall to several SMs is
- * finished by the last of them, which merges the partial results
- * (log-sum-exp rule) from the workspace.
+ * Decode with the batch's cached tokens divided evenly among the SMs: the same
+ * result as gqa_decode_rows (same arguments, same row check, same device
+ * status), built for groups of many query heads per KV head (MQA, wide GQA)
+ * and for ragged lengths.  Per byte of K/V a group of h / n_kv heads does
+ * h / n_kv multiply-adds for each product ("Multi-query attention"
+ * (pranaymahendrakar), "Why this is a bandwidth argument, not a FLOP
+ * argument"), and a fixed number of splits per sequence leaves SMs idle
+ * while the longest sequences finish; here the tokens of the whole batch are
+ * laid end to end and each SM's CTAs take an equal share, whatever the
+ * sequence boundaries.  By group size (as measured): 17 to 64 heads at
+ * d_h = 128 run warp-level MMAs, two CTAs per SM; smaller groups at
+ * d_h = 128 run tcgen05 products with the tokens as the rows; d_h = 64 and
+ * groups above 64 heads run tcgen05 products with the heads as the rows (a
+ * group of at most 64 (32) heads as 2 (4) copies, each over its own share of
+ * every stage's tokens).  The pieces of a sequence that fell to several CTAs
+ * are merged (log-sum-exp rule) from the workspace by a second kernel.
  *   workspace        DEVICE memory of at least
  *                    gqa_decode_split_workspace_bytes(B, h, n_kv, d_h) bytes
  *                    (which depends on the current device's SM count),
@@ -175,8 +180,10 @@ size_t gqa_decode_split_workspace_bytes(int B, int h, int n_kv, int d_h);
  * Errors: as gqa_decode_split (without the workspace checks), plus
  * GQA_ERR_UNSUPPORTED when the sizes need more than the 16 MiB array, that is
  * when gqa_decode_split_workspace_bytes(B, h, n_kv, d_h) exceeds 16 MiB (on a
- * 148-SM B200: n_kv * ceil(h / n_kv / 128) * B above 104 at d_h = 128, above
- * 348 at d_h = 64), and GQA_ERR_CUDA if the address lookup or a launch fails.
+ * 148-SM B200: n_kv * B above 208 for 17 to 64 query heads per KV head at
+ * d_h = 128; otherwise n_kv * ceil(h / n_kv / 128) * B above 104 at
+ * d_h = 128, above 348 at d_h = 64), and GQA_ERR_CUDA if the address lookup
+ * or a launch fails.
  * Nothing is launched on an argument or size error.
  */
 int gqa_decode_split_noalloc(const void *q, const void *k_cache, const void *v_cache, int64_t cache_rows,

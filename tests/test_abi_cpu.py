@@ -196,3 +196,17 @@ def test_wait_test_library_exports_everything():
     # the product library has no test hook
     with pytest.raises(AttributeError):
         getattr(gqa.lib(), "gqa_test_set_stall")
+
+
+def test_decode_dispatch_rule_on_cpu():
+    """decode()'s choice of the split path for mid-sized groups at d = 128 (the branches
+    that need no device query)."""
+    import torch
+    from attention_gqa_decode_b200 import _lib as L
+    q = torch.zeros(64, 32, 128)
+    k = torch.zeros(64 * 8192, 1, 128)
+    assert L.use_split(q, k)                               # MQA, 32 heads per KV head
+    assert L.use_split(torch.zeros(4, 64, 128), torch.zeros(4 * 300, 1, 128))
+    assert not L.use_split(torch.zeros(4, 64, 128), torch.zeros(4 * 100, 1, 128))   # too few rows per sequence
+    assert L.use_split(torch.zeros(4, 96, 128), torch.zeros(4 * 300, 2, 128))   # 48 heads per KV head
+    assert not L.use_split(torch.zeros(4, 30, 128), torch.zeros(4 * 300, 4, 128))  # h % n_kv != 0

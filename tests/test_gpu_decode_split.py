@@ -1,5 +1,8 @@
-"""gqa_decode_split (the batch's tokens divided evenly among the SMs, tensor-core
-products, partial results merged through the workspace) against the fp64 oracle.
+"""gqa_decode_split (the batch's tokens divided evenly among the SMs, partial results
+merged through the workspace) against the fp64 oracle.  By group size it runs the
+tokens-as-rows tcgen05 kernel (up to 16 heads, d = 128), the balanced warp-level kernel
+(17 to 64 heads, d = 128; two token groups per m-tile up to 32 heads) or the heads-as-rows
+tcgen05 kernel (d = 64; and above 64 heads, with 2 or 4 copies of small groups at d = 64).
 
 The kernel cuts sequences at arbitrary token positions, so the cases aim at
 the places a cut can fall: lengths around the 64-token stage, sequences
@@ -127,6 +130,9 @@ def test_decode_dispatch():
     assert torch.equal(gqa.decode(q, k, v, lens), gqa.decode_split(q, k, v, lens))
     q, k, v, lens = (t.cuda() for t in inputs.decode_inputs(38, 16, 64, 8, 128, 300))   # the GQA shape
     assert not _lib.use_split(q, k)
+    q, k, v, lens = (t.cuda() for t in inputs.decode_inputs(38, 64, 32, 1, 128, 600))   # MQA: the balanced kernel
+    assert _lib.use_split(q, k)
+    assert torch.equal(gqa.decode(q, k, v, lens), gqa.decode_split(q, k, v, lens))
 
 
 def test_split_status_clean():

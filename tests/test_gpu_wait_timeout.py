@@ -150,10 +150,11 @@ def test_product_library_status_clean():
     assert gqa.gqa_get_device_status() == _lib.GQA_OK
 
 
-@pytest.mark.parametrize("B,h,n_kv,d", [(6, 64, 1, 128), (3, 128, 1, 128), (4, 32, 2, 64)], ids=str)
+@pytest.mark.parametrize("B,h,n_kv,d", [(6, 64, 1, 128), (5, 32, 1, 128), (3, 128, 1, 128), (4, 32, 2, 64)], ids=str)
 def test_split_decode_wait_runs_out(W, B, h, n_kv, d):
-    """The split-KV kernels (and their merge): the stalled call times out, and the next
-    call through the same workspace is exact."""
+    """The split-KV kernels (balanced warp-level with one and two token groups,
+    heads-as-rows at d = 128 and 64, and their merge): the stalled call times out, and
+    the next call through the same workspace is exact."""
     q, k, v, L = (t.cuda() for t in inputs.decode_inputs(27, B, h, n_kv, d, [3000, 10, 700, 5000, 64, 1][:B]))
     out = torch.empty_like(q)
     nbytes = W.gqa_decode_split_workspace_bytes(B, h, n_kv, d)
