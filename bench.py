@@ -57,6 +57,14 @@ def peaks():
         return {"hbm": FALLBACK_HBM_GBS, "bf16": FALLBACK_BF16_TFLOPS, "bf16_sustained": 1400.0, "src": "fallback"}
 
 
+# the committed ncu traffic record of the decode launch each named leg times (the split
+# path's merge kernel is not included: 5.9 MB of L2-resident partials at MQA B64)
+NAMED_TRAFFIC = {"decode_mqa": "gqa_decode_bal_kernel[mqa]",
+                 "decode_ragged_nkv64": "gqa_decode_kernel[ragged n_kv64]",
+                 "decode_ragged_nkv8": "gqa_decode_kernel[ragged n_kv8]",
+                 "decode_ragged_nkv1": "gqa_decode_bal_kernel[ragged n_kv1]"}
+
+
 def kernel_traffic(kernel: str):
     """DRAM bytes per launch from the committed ncu summary, if its source hash is current."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -619,7 +627,7 @@ def main():
             "kv_bytes_per_decoded_token": r["bytes_per_token"],
             "l2": f"{r['copies']} cache copies rotated",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm"], "traffic": None,
+                         "frac": gbs / pk["hbm"], "traffic": kernel_traffic(NAMED_TRAFFIC.get(name, "")),
                          "algorithmic_bytes_per_launch": r["kv_bytes"], "peak_source": pk["src"]}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"], parity = oracle_decode_leg(target_s=10.0, gpu_out=dec["out"])
