@@ -28,7 +28,7 @@ def run(q, k, v, lens, scale=None):
     return out.cpu()
 
 
-@pytest.mark.parametrize("G", [1, 4, 8, 16, 32, 48, 64, 128, 192])
+@pytest.mark.parametrize("G", [1, 4, 8, 16, 17, 24, 32, 40, 48, 56, 64, 96, 128, 192])
 @pytest.mark.parametrize("d", [64, 128])
 def test_split_group_sizes(G, d):
     n_kv = 2
