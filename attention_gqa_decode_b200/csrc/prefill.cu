@@ -144,6 +144,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
+    // the short-row pairs' launch (SPLIT, queued behind this one) may start on SMs this
+    // launch's last wave leaves idle: the two write disjoint rows
+    if constexpr (!SPLIT && !PAGED) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     // work unit: heaviest causal query-tile pairs first; consecutive CTAs share a KV group
@@ -545,6 +548,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
     }
 
+    // a short-row launch that started beside the common one finishes only after it, so that
+    // work queued behind this launch still sees every output row
+    if constexpr (SPLIT && !PAGED) asm volatile("griddepcontrol.wait;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     if (warp == 9) {
@@ -637,6 +643,22 @@ static int launch_prefill_range(const PrefillCall &c, int pair_lo, int pair_hi) 
     const long ctas = static_cast<long>(pair_hi - pair_lo) * c.B * c.h;
     if (ctas <= 0) return 0;
     if (ctas > 0x7fffffffL) return 1;
+    if constexpr (SPLIT && !PAGED) {
+        // a programmatic dependent of the common launch just queued (a plain launch where the
+        // attribute is refused: the kernel's final wait is then a no-op)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
+        cfg.blockDim = dim3(kPfThreads, 1, 1);
+        cfg.dynamicSmemBytes = SM::kTotal;
+        cfg.stream = c.stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, tkp, tvp, prm) == cudaSuccess) return 0;
+        (void)cudaGetLastError();
+    }
     kern<<<static_cast<unsigned>(ctas), kPfThreads, SM::kTotal, c.stream>>>(tq, tk, tv, tkp, tvp, prm);
     return cudaGetLastError() == cudaSuccess ? 0 : 3;
 }
