@@ -52,6 +52,7 @@
 // instantiation (SPLIT), launched only for the query-tile pairs that need it,
 // so the common path is compiled without it.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -416,112 +417,125 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             split = first_row_keys(PAGED, p.causal, p.S_q, p.S_kv, q0 + t * kPfRows, past) <= kPfSplitKeys;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < n_t; ++j) {
-            const bool landed = mbar_wait(&sfull[t], j & 1, abort_flag, p.status);
-            if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }   // tcgen05.ld/st are warp-aligned
-            tc_fence_after();
-            // the whole S row of this thread, read once.  Columns c <= lim_c are visible:
-            // PAGED past tile: cached tokens below `past`; chunk tile: causal within the chunk
-            const int lim_c = !PAGED ? limit - j * kPfKeys
-                              : j < n_past ? past - 1 - j * kPfKeys
-                                           : row - (j - n_past) * kPfKeys;
-            const bool masked = lim_c < kPfKeys - 1;
-            static_assert(kPfKeys == 128, "four 32-column TMEM loads per row");
-            uint32_t r0[32], r1[32], r2[32], r3[32];
-            tmem_ld32(tS, r0);
-            tmem_ld32(tS + 32, r1);
-            tmem_ld32(tS + 64, r2);
-            tmem_ld32(tS + 96, r3);
-            tmem_wait_ld();
-            // column c of the row (c is a compile-time constant after unrolling)
-#define GQA_S(c) ((c) < 32 ? r0[(c)] : (c) < 64 ? r1[(c) - 32] : (c) < 96 ? r2[(c) - 64] : r3[(c) - 96])
-            float mx;
-            if (!masked) {
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int c = 0; c < kPfKeys; c += 8) {
-                    m4[0] = fmax3(m4[0], __uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)));
-                    m4[1] = fmax3(m4[1], __uint_as_float(GQA_S(c + 2)), __uint_as_float(GQA_S(c + 3)));
-                    m4[2] = fmax3(m4[2], __uint_as_float(GQA_S(c + 4)), __uint_as_float(GQA_S(c + 5)));
-                    m4[3] = fmax3(m4[3], __uint_as_float(GQA_S(c + 6)), __uint_as_float(GQA_S(c + 7)));
-                }
-                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            } else {
-                mx = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < kPfKeys; ++c)
-                    if (c <= lim_c) mx = fmaxf(mx, __uint_as_float(GQA_S(c)));
-            }
-            const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * cl2;
-            if (j == 0) {
-                m_used = m_tile;
-            } else {
-                const bool need = m_tile > m_used + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, need)) {
-                    const float m_new = need ? m_tile : m_used;
-                    const float alpha = exp2f(m_used - m_new);
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t ro[32];
-                        tmem_ld32(tO + c * 32, ro);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
-                        tmem_st32(tO + c * 32, ro);
+        // the key-tile loop; the SPLIT instantiation compiles it twice (with the remainder pass
+        // and without) and picks one per query tile, so the loop that runs stays compact
+        auto tile_loop = [&](auto rem_tag) {
+            constexpr bool kRem = decltype(rem_tag)::value;
+            for (int j = 0; j < n_t; ++j) {
+                const bool landed = mbar_wait(&sfull[t], j & 1, abort_flag, p.status);
+                if (!__all_sync(0xffffffffu, landed)) { ok = false; break; }   // tcgen05.ld/st are warp-aligned
+                tc_fence_after();
+                // the whole S row of this thread, read once.  Columns c <= lim_c are visible:
+                // PAGED past tile: cached tokens below `past`; chunk tile: causal within the chunk
+                const int lim_c = !PAGED ? limit - j * kPfKeys
+                                  : j < n_past ? past - 1 - j * kPfKeys
+                                               : row - (j - n_past) * kPfKeys;
+                const bool masked = lim_c < kPfKeys - 1;
+                static_assert(kPfKeys == 128, "four 32-column TMEM loads per row");
+                uint32_t r0[32], r1[32], r2[32], r3[32];
+                tmem_ld32(tS, r0);
+                tmem_ld32(tS + 32, r1);
+                tmem_ld32(tS + 64, r2);
+                tmem_ld32(tS + 96, r3);
+                tmem_wait_ld();
+                // column c of the row (c is a compile-time constant after unrolling)
+    #define GQA_S(c) ((c) < 32 ? r0[(c)] : (c) < 64 ? r1[(c) - 32] : (c) < 96 ? r2[(c) - 64] : r3[(c) - 96])
+                float mx;
+                if (!masked) {
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    #pragma unroll
+                    for (int c = 0; c < kPfKeys; c += 8) {
+                        m4[0] = fmax3(m4[0], __uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)));
+                        m4[1] = fmax3(m4[1], __uint_as_float(GQA_S(c + 2)), __uint_as_float(GQA_S(c + 3)));
+                        m4[2] = fmax3(m4[2], __uint_as_float(GQA_S(c + 4)), __uint_as_float(GQA_S(c + 5)));
+                        m4[3] = fmax3(m4[3], __uint_as_float(GQA_S(c + 6)), __uint_as_float(GQA_S(c + 7)));
                     }
-                    tmem_wait_st();
-                    l *= alpha;
-                    m_used = m_new;
+                    mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                } else {
+                    mx = -INFINITY;
+    #pragma unroll
+                    for (int c = 0; c < kPfKeys; ++c)
+                        if (c <= lim_c) mx = fmaxf(mx, __uint_as_float(GQA_S(c)));
                 }
-            }
-            // P = exp2(S * scale * log2(e) - m) as packed bf16, written back over S;
-            // the running sum adds exactly the rounded weights P V uses
-            float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            if (SPLIT && split) {   // first the remainders w - bf16(w) (exact in fp32), as bf16, over
-                                    // the upper half of S (its scores are in registers already)
-#pragma unroll
-                for (int ch = 0; ch < kPfKeys / 16; ++ch) {
-                    uint32_t rk[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int c = ch * 16 + 2 * e;
-                        const float2 x =
-                            ffma2_bcast(__uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)), cl2, -m_used);
-                        float w0 = exp2f(x.x), w1 = exp2f(x.y);
-                        if (masked) {
-                            if (c > lim_c) w0 = 0.f;
-                            if (c + 1 > lim_c) w1 = 0.f;
+                const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * cl2;
+                if (j == 0) {
+                    m_used = m_tile;
+                } else {
+                    const bool need = m_tile > m_used + kRescaleThreshold;
+                    if (__any_sync(0xffffffffu, need)) {
+                        const float m_new = need ? m_tile : m_used;
+                        const float alpha = exp2f(m_used - m_new);
+    #pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t ro[32];
+                            tmem_ld32(tO + c * 32, ro);
+                            tmem_wait_ld();
+    #pragma unroll
+                            for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
+                            tmem_st32(tO + c * 32, ro);
                         }
-                        const float2 u = unpack_bf16x2(pack_bf16x2(w0, w1));
-                        rk[e] = pack_bf16x2(w0 - u.x, w1 - u.y);
-                        rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(rk[e]));
+                        tmem_wait_st();
+                        l *= alpha;
+                        m_used = m_new;
                     }
-                    tmem_st8(tS + kPfKeys / 2 + ch * 8, rk);
                 }
-            }
-#pragma unroll
-            for (int ch = 0; ch < kPfKeys / 32; ++ch) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int c = ch * 32 + 2 * e;
-                    const float2 x = ffma2_bcast(__uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)), cl2, -m_used);
-                    uint32_t pp = pack_bf16x2(exp2f(x.x), exp2f(x.y));
-                    if (masked) {   // masked keys add nothing (also when scale == 0)
-                        if (c > lim_c) pp &= 0xFFFF0000u;
-                        if (c + 1 > lim_c) pp &= 0x0000FFFFu;
+                // P = exp2(S * scale * log2(e) - m) as packed bf16, written back over S;
+                // the running sum adds exactly the rounded weights P V uses
+                float2 rs2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                if constexpr (kRem) {   // first the remainders w - bf16(w) (exact in fp32), as bf16, over
+                                        // the upper half of S (its scores are in registers already)
+    #pragma unroll
+                    for (int ch = 0; ch < kPfKeys / 16; ++ch) {
+                        uint32_t rk[8];
+    #pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int c = ch * 16 + 2 * e;
+                            const float2 x =
+                                ffma2_bcast(__uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)), cl2, -m_used);
+                            float w0 = exp2f(x.x), w1 = exp2f(x.y);
+                            if (masked) {
+                                if (c > lim_c) w0 = 0.f;
+                                if (c + 1 > lim_c) w1 = 0.f;
+                            }
+                            const float2 u = unpack_bf16x2(pack_bf16x2(w0, w1));
+                            rk[e] = pack_bf16x2(w0 - u.x, w1 - u.y);
+                            rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(rk[e]));
+                        }
+                        tmem_st8(tS + kPfKeys / 2 + ch * 8, rk);
                     }
-                    pk[e] = pp;
-                    rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(pp));
                 }
-                tmem_st16(tS + ch * 16, pk);
+    #pragma unroll
+                for (int ch = 0; ch < kPfKeys / 32; ++ch) {
+                    uint32_t pk[16];
+    #pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int c = ch * 32 + 2 * e;
+                        const float2 x = ffma2_bcast(__uint_as_float(GQA_S(c)), __uint_as_float(GQA_S(c + 1)), cl2, -m_used);
+                        uint32_t pp = pack_bf16x2(exp2f(x.x), exp2f(x.y));
+                        if (masked) {   // masked keys add nothing (also when scale == 0)
+                            if (c > lim_c) pp &= 0xFFFF0000u;
+                            if (c + 1 > lim_c) pp &= 0x0000FFFFu;
+                        }
+                        pk[e] = pp;
+                        rs2[e & 1] = fadd2(rs2[e & 1], unpack_bf16x2(pp));
+                    }
+                    tmem_st16(tS + ch * 16, pk);
+                }
+    #undef GQA_S
+                const float rs = (rs2[0].x + rs2[1].x) + (rs2[0].y + rs2[1].y);
+                l += rs;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&pfull[t]);
             }
-#undef GQA_S
-            const float rs = (rs2[0].x + rs2[1].x) + (rs2[0].y + rs2[1].y);
-            l += rs;
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&pfull[t]);
+        };
+        if constexpr (SPLIT) {
+            if (split)
+                tile_loop(std::true_type{});
+            else
+                tile_loop(std::false_type{});
+        } else {
+            tile_loop(std::false_type{});
         }
         // epilogue: O / l -> bf16 -> out[b, row, head, :]
         const bool fin = n_t > 0 && ok && mbar_wait(&odone[t], 0, abort_flag, p.status);

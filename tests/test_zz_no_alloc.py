@@ -30,8 +30,9 @@ def _noalloc(q, k, v, lens, out):
 
 
 @pytest.mark.parametrize("B,h,n_kv,d,lens", [
-    (6, 64, 1, 128, [3000, 10, 700, 5000, 64, 1]),
-    (4, 32, 2, 64, [129, 2000, 0, 333]),
+    (6, 64, 1, 128, [3000, 10, 700, 5000, 64, 1]),     # 64 heads per KV head: balanced, one token group
+    (5, 32, 1, 128, [4000, 17, 900, 0, 2500]),         # 32: balanced, two token groups
+    (4, 32, 2, 64, [129, 2000, 0, 333]),               # d 64: heads as the MMA rows
 ], ids=str)
 def test_noalloc_matches_the_workspace_entry_point_twice(B, h, n_kv, d, lens):
     q, k, v, L = (t.cuda() for t in inputs.decode_inputs(41 + d, B, h, n_kv, d, lens))
@@ -56,3 +57,15 @@ def test_noalloc_rejects_sizes_beyond_its_array():
     torch.cuda.synchronize()
     assert torch.all(out == 0)                     # nothing launched
     assert np.isfinite(out.float().cpu().numpy()).all()
+
+
+def test_noalloc_rejects_a_balanced_shape_beyond_its_array():
+    # 32 heads per KV head at d 128: 296 CTA slots + one per (KV head, sequence), 33 KB each
+    B, h, n_kv, d = 256, 32, 1, 128
+    assert gqa.gqa_decode_split_workspace_bytes(B, h, n_kv, d) > 16 << 20
+    assert gqa.gqa_decode_split_workspace_bytes(200, h, n_kv, d) <= 16 << 20
+    q, k, v, L = (t.cuda() for t in inputs.decode_inputs(44, B, h, n_kv, d, 8))
+    out = torch.zeros_like(q)
+    assert _noalloc(q, k, v, L, out) == _lib.GQA_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
