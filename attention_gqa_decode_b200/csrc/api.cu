@@ -174,6 +174,7 @@ int gqa_decode_rows(const void *q, const void *k_cache, const void *v_cache, int
 
 size_t gqa_decode_split_workspace_bytes(int B, int h, int n_kv, int d_h) {
     if (B <= 0 || B > 65535 || h <= 0 || n_kv <= 0 || h % n_kv != 0 || (d_h != 64 && d_h != 128)) return 0;
+    if (static_cast<long long>(n_kv) * ((h / n_kv + 127) / 128) * B > (1LL << 24)) return 0;   // as gqa_decode_split
     return gqa::split_workspace_bytes(B, h, n_kv, d_h);
 }
 

@@ -210,3 +210,13 @@ def test_decode_dispatch_rule_on_cpu():
     assert not L.use_split(torch.zeros(4, 64, 128), torch.zeros(4 * 100, 1, 128))   # too few rows per sequence
     assert L.use_split(torch.zeros(4, 96, 128), torch.zeros(4 * 300, 2, 128))   # 48 heads per KV head
     assert not L.use_split(torch.zeros(4, 30, 128), torch.zeros(4 * 300, 4, 128))  # h % n_kv != 0
+
+
+@pytest.mark.parametrize("B,h,n_kv,d", [
+    (0, 32, 1, 128), (70000, 32, 1, 128), (4, 30, 4, 128), (4, 32, 0, 128), (4, 32, 1, 96),
+    (65535, 512, 512, 128),   # 33.5 M (KV head, sequence) segments: past the split decode's 2^24
+], ids=str)
+def test_split_workspace_bytes_is_zero_for_rejected_sizes(L, B, h, n_kv, d):
+    """gqa_decode_split_workspace_bytes answers 0 exactly where gqa_decode_split refuses the sizes
+    (these cases return before the device's SM count is looked up)."""
+    assert L.gqa_decode_split_workspace_bytes(B, h, n_kv, d) == 0
