@@ -227,3 +227,23 @@ def test_mla_and_fp8_lengths_past_the_cache_rows_are_cut_and_reported():
     ref = oracle.decode_general(q, kc, vc, torch.tensor([300, 150], dtype=torch.int32), fp8=True, k_scale=ks,
                                 v_scale=vs)
     check(got, ref, "E4M3 cut", v=vc, v_scale=vs, n_keys=300)
+
+
+def test_prefill_output_is_complete_for_work_queued_behind_it():
+    """A causal prefill is two launches (the common query-tile pairs, then the pairs whose
+    rows see few keys, started beside the first one's last wave).  Work queued behind the
+    call on the same stream must see every output row: copy the output on that stream,
+    before any host synchronisation, and compare the copy with the oracle."""
+    B, S, h, n_kv, d = 2, 1024, 8, 2, 128
+    q, k, v = inputs.prefill_inputs(61, B, S, S, h, n_kv, d)
+    ref = oracle.prefill(q, k, v, causal=True)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            out = torch.full_like(qd, float("nan"))
+            got = gqa.prefill(qd, kd, vd, causal=True, out=out)
+            snap = got.clone()                     # queued on `side`, behind both launches
+            side.synchronize()
+            assert torch.isfinite(snap.float()).all()
+            check(snap.cpu(), ref, "prefill output copied on the same stream", v=v, n_keys=S)
