@@ -410,27 +410,59 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
         }
         return;
     }
+    // this CTA combines rows split, split + P, ...: first each row's weights over the splits
+    // (into the partial-score area, which no peer reads), then the rows, with every split's
+    // float4 loaded at once
+    float *wn = reinterpret_cast<float *>(sred);   // [row][kMlaMaxSplit]
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     const int nrows = (HS - split + P - 1) / P;
-    for (int it = threadIdx.x; it < nrows * (kMlaDc / 2); it += kMlaThreads) {
-        const int r = split + P * (it / (kMlaDc / 2)), c = 2 * (it % (kMlaDc / 2));
+    for (int k = threadIdx.x; k < nrows; k += kMlaThreads) {
+        const int r = split + P * k;
+        float mq[kMlaMaxSplit], lq[kMlaMaxSplit];
         float M = -INFINITY;
-        for (int q = 0; q < P; ++q) M = fmaxf(M, *cluster.map_shared_rank(&cm[r], q));
-        float sl = 0.f, s0 = 0.f, s1 = 0.f;
-        if (M != -INFINITY) {
-            for (int q = 0; q < P; ++q) {
-                const float mq = *cluster.map_shared_rank(&cm[r], q);
-                if (mq == -INFINITY) continue;   // a split with no tokens
-                const float w = exp2f(mq - M);
-                sl += w * *cluster.map_shared_rank(&cl[r], q);
-                const float2 v = *reinterpret_cast<const float2 *>(cluster.map_shared_rank(&co[r * kMlaDc + c], q));
-                s0 += w * v.x;
-                s1 += w * v.y;
-            }
+#pragma unroll
+        for (int q = 0; q < kMlaMaxSplit; ++q) {
+            mq[q] = q < P ? *cluster.map_shared_rank(&cm[r], q) : -INFINITY;
+            lq[q] = q < P ? *cluster.map_shared_rank(&cl[r], q) : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < kMlaMaxSplit; ++q) M = fmaxf(M, mq[q]);
+        float sl = 0.f;
+#pragma unroll
+        for (int q = 0; q < kMlaMaxSplit; ++q) {
+            mq[q] = (M == -INFINITY || mq[q] == -INFINITY) ? 0.f : exp2f(mq[q] - M);   // a split with no tokens adds nothing
+            sl += mq[q] * lq[q];
         }
         const float inv = sl > 0.f ? 1.f / sl : 0.f;
-        if (ok) *reinterpret_cast<__nv_bfloat162 *>(ob + r * kMlaDc + c) = __floats2bfloat162_rn(s0 * inv, s1 * inv);
+#pragma unroll
+        for (int q = 0; q < kMlaMaxSplit; ++q) wn[k * kMlaMaxSplit + q] = mq[q] * inv;
+    }
+    __syncthreads();
+    for (int it = threadIdx.x; it < nrows * (kMlaDc / 4); it += kMlaThreads) {
+        const int k = it / (kMlaDc / 4), c = 4 * (it % (kMlaDc / 4));
+        const int r = split + P * k;
+        float4 v[kMlaMaxSplit];
+#pragma unroll
+        for (int q = 0; q < kMlaMaxSplit; ++q)
+            if (q < P) v[q] = *reinterpret_cast<const float4 *>(cluster.map_shared_rank(&co[r * kMlaDc + c], q));
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < kMlaMaxSplit; ++q)
+            if (q < P) {
+                const float w = wn[k * kMlaMaxSplit + q];
+                a.x += w * v[q].x;
+                a.y += w * v[q].y;
+                a.z += w * v[q].z;
+                a.w += w * v[q].w;
+            }
+        if (ok) {
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<const uint32_t *>(&lo);
+            pk.y = *reinterpret_cast<const uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(ob + static_cast<size_t>(r) * kMlaDc + c) = pk;
+        }
     }
     cluster.sync();
 }
