@@ -29,6 +29,7 @@ SIGNATURES = {
     "gqa_prefill_paged": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_mla_decode": ([_vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp], _i),
     "gqa_mla_decode_rows": ([_vp, _vp, _i64, _vp, _vp, _i, _i, _i, _f, _vp], _i),
+    "gqa_mla_decode_path": ([_i, _i, _i, _i64], _i),
     "gqa_status_string": ([_i], ctypes.c_char_p),
     "gqa_get_device_status": ([_vp], _i),
 }
@@ -109,6 +110,10 @@ def gqa_decode_fp8_rows(q, k_cache, v_cache, cache_rows, k_scale, v_scale, seqle
 
 def gqa_mla_decode_rows(q_absorbed, c_kv, cache_rows, seqlens, out, B, h, d_c, scale, stream) -> int:
     return lib().gqa_mla_decode_rows(q_absorbed, c_kv, int(cache_rows), seqlens, out, B, h, d_c, float(scale), stream)
+
+
+def gqa_mla_decode_path(B, h, d_c, cache_rows) -> int:
+    return lib().gqa_mla_decode_path(B, h, d_c, int(cache_rows))
 
 
 def gqa_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, B, h, n_kv, d_h, scale, stream) -> int:

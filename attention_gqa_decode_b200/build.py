@@ -20,7 +20,7 @@ from concurrent.futures import ThreadPoolExecutor
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["api.cu", "decode.cu", "decode_split.cu", "prefill.cu", "mla.cu"]
+SOURCES = ["api.cu", "decode.cu", "decode_split.cu", "prefill.cu", "mla.cu", "mla_tc.cu"]
 HEADERS = ["common.cuh"]
 LIB = os.path.join(PKG, "libgqa_b200.so")
 WAITTEST_LIB = os.path.join(PKG, "libgqa_b200_waittest.so")

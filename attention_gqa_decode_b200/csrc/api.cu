@@ -27,7 +27,8 @@ int launch_prefill_paged(const void *q, const void *k_new, const void *v_new, vo
                          const int32_t *past_lens, void *out, int B, int S_q, int h, int n_kv, int d, float scale,
                          cudaStream_t stream);
 int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h, float scale,
-                      long long cache_rows, cudaStream_t stream);
+                      long long cache_rows, bool rows_known, cudaStream_t stream);
+bool mla_prefers_tc(int B, int h, long long cache_rows, bool rows_known, int sms);
 int launch_decode_ex(const void *q, const void *k, const void *v, const float *k_scale, const float *v_scale,
                      const int32_t *seqlens, const int32_t *block_table, int max_blocks, int page_size,
                      int num_pages, void *out, int B, int h, int n_kv, int d, float scale, long long cache_rows,
@@ -309,26 +310,31 @@ int gqa_prefill_paged(const void *q, const void *k_new, const void *v_new, void 
                                      num_pages, past_lens, out, B, S_q, h, n_kv, d_h, scale, stream);
 }
 
-static int mla_decode(const void *q_absorbed, const void *c_kv, long long cache_rows, const int32_t *seqlens,
-                      void *out, int B, int h, int d_c, float scale, cudaStream_t stream) {
+static int mla_decode(const void *q_absorbed, const void *c_kv, long long cache_rows, bool rows_known,
+                      const int32_t *seqlens, void *out, int B, int h, int d_c, float scale, cudaStream_t stream) {
     if (!q_absorbed || !c_kv || !seqlens || !out) return GQA_ERR_INVALID_ARG;
     if (!aligned16(q_absorbed) || !aligned16(c_kv) || !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
         return GQA_ERR_INVALID_ARG;
     if (B <= 0 || B > 65535 || h <= 0 || h > 65535 * 16) return GQA_ERR_INVALID_ARG;
     if (!scale_ok(scale)) return GQA_ERR_INVALID_ARG;
     if (d_c != 512) return GQA_ERR_UNSUPPORTED;
-    return gqa::launch_mla_decode(q_absorbed, c_kv, seqlens, out, B, h, scale, cache_rows, stream);
+    return gqa::launch_mla_decode(q_absorbed, c_kv, seqlens, out, B, h, scale, cache_rows, rows_known, stream);
 }
 
 int gqa_mla_decode(const void *q_absorbed, const void *c_kv, const int32_t *seqlens, void *out, int B, int h,
                    int d_c, float scale, cudaStream_t stream) {
-    return mla_decode(q_absorbed, c_kv, kOpenRows, seqlens, out, B, h, d_c, scale, stream);
+    return mla_decode(q_absorbed, c_kv, kOpenRows, false, seqlens, out, B, h, d_c, scale, stream);
 }
 
 int gqa_mla_decode_rows(const void *q_absorbed, const void *c_kv, int64_t cache_rows, const int32_t *seqlens,
                         void *out, int B, int h, int d_c, float scale, cudaStream_t stream) {
     if (!rows_ok(cache_rows)) return GQA_ERR_INVALID_ARG;
-    return mla_decode(q_absorbed, c_kv, cache_rows, seqlens, out, B, h, d_c, scale, stream);
+    return mla_decode(q_absorbed, c_kv, cache_rows, true, seqlens, out, B, h, d_c, scale, stream);
+}
+
+int gqa_mla_decode_path(int B, int h, int d_c, int64_t cache_rows) {
+    if (B <= 0 || h <= 0 || d_c != 512 || !rows_ok(cache_rows)) return -1;
+    return gqa::mla_prefers_tc(B, h, cache_rows, true, gqa_host::sm_count()) ? 1 : 0;
 }
 
 const char *gqa_status_string(int status) {

@@ -470,8 +470,29 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
 // ---------------------------------------------------------------------------
 // host launcher
 
+int launch_mla_decode_tc(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h,
+                         float scale, long long cache_rows, cudaStream_t stream);
+
+// The tensor-core kernel (mla_tc.cu) for long sequences in batches too small to
+// fill the GPU with this kernel: more than 16 heads (its products are 32 heads
+// wide), this kernel's CTAs (16-head groups x up to 8 splits) fewer than the
+// SMs, and, by the caller's row count, at least kMlaTcMinAvgRows tokens per
+// sequence on average.  Measured on B200 (us, this kernel / tensor cores):
+// B8 h32 L32768 208 / 168, B1 h32 L20000 109 / 73; it loses where this kernel
+// fills the SMs (B16 h32 L4096 34 / 46) or on short or 16-head work.
+constexpr long long kMlaTcMinAvgRows = 8192;
+
+bool mla_prefers_tc(int B, int h, long long cache_rows, bool rows_known, int sms) {
+    if (!rows_known || h <= kMlaHeads) return false;
+    const long units = static_cast<long>(B) * ((h + kMlaHeads - 1) / kMlaHeads);
+    const long P = std::max(1L, std::min(static_cast<long>(kMlaMaxSplit), 2L * sms / units));
+    return units * P < sms && cache_rows >= kMlaTcMinAvgRows * B;
+}
+
 int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h, float scale,
-                      long long cache_rows, cudaStream_t stream) {
+                      long long cache_rows, bool rows_known, cudaStream_t stream) {
+    if (mla_prefers_tc(B, h, cache_rows, rows_known, gqa_host::sm_count()))
+        return launch_mla_decode_tc(q, c_kv, seqlens, out, B, h, scale, cache_rows, stream);
     auto kern = gqa_mla_decode_kernel;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 3;

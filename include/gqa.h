@@ -312,10 +312,22 @@ int gqa_mla_decode(const void *q_absorbed, const void *c_kv, const int32_t *seql
                    int B, int h, int d_c, float scale, cudaStream_t stream);
 
 /* gqa_mla_decode over a latent cache of `cache_rows` rows, with the row check
- * of gqa_decode_rows (lengths past the cache cut and reported). */
+ * of gqa_decode_rows (lengths past the cache cut and reported).  With the row
+ * count known, long sequences in small batches run on a second kernel (see
+ * gqa_mla_decode_path); the results agree within the same bound. */
 int gqa_mla_decode_rows(const void *q_absorbed, const void *c_kv, int64_t cache_rows,
                         const int32_t *seqlens, void *out,
                         int B, int h, int d_c, float scale, cudaStream_t stream);
+
+/* Which kernel gqa_mla_decode_rows runs for a shape on the current device:
+ * 0 = warp-level MMA (16-head groups, splits of one sequence merged in a
+ * thread-block cluster; gqa_mla_decode always runs it), 1 = 5th-generation
+ * tensor cores (32-head groups, q' resident in tensor memory, one CTA per SM),
+ * taken when h > 16, the warp-level kernel's CTAs (B * ceil(h / 16) times up
+ * to 8 splits) are fewer than the SMs, and cache_rows >= 8192 * B.  Host-only
+ * (reads the SM count; 148 when no device answers).  Returns -1 for B <= 0,
+ * h <= 0, d_c != 512 or cache_rows outside [0, 2^31). */
+int gqa_mla_decode_path(int B, int h, int d_c, int64_t cache_rows);
 
 /* A static, human-readable name for a gqa_status_t value. */
 const char *gqa_status_string(int status);

@@ -26,6 +26,10 @@ def run(q, c, lens, scale=None):
     (3, 40, [64, 0, 7]),             # a partial head group, an empty sequence
     (1, 32, [20000]),                # long: eight splits
     (1, 96, [9000]),                 # several head groups, several splits each
+    # long sequences in small batches: the tensor-core kernel (asserted below)
+    (2, 32, [0, 17000]),             # an empty sequence
+    (3, 40, [9000, 255, 30000]),     # a partial 32-head group; a short sequence (remainder product)
+    (4, 64, [8192, 1, 64, 40000]),   # one token; exactly one stage
 ], ids=str)
 def test_mla_parity(B, h, lens):
     q, c, lens = inputs.mla_decode_inputs(60 + h, B, h, 512, lens)
@@ -84,3 +88,37 @@ def spiked_inputs(seed, B, h, lens):
 def test_mla_running_max_rescale():
     q, c, lens = spiked_inputs(70, 3, 32, [1000, 300, 2049])
     check(run(q, c, lens), oracle.mla_decode(q, c, lens), "MLA with rescales", v=c, n_keys=2049)
+
+
+def tc_path(B, h, lens):
+    return gqa.gqa_mla_decode_path(B, h, 512, int(sum(max(x, 0) for x in lens)))
+
+
+def test_mla_cases_cover_both_kernels():
+    assert tc_path(1, 32, [20000]) == 1 and tc_path(1, 96, [9000]) == 1 and tc_path(2, 32, [0, 17000]) == 1
+    assert tc_path(3, 40, [9000, 255, 30000]) == 1 and tc_path(4, 64, [8192, 1, 64, 40000]) == 1
+    assert tc_path(3, 32, [1, 31, 33]) == 0 and tc_path(16, 32, [4096] * 16) == 0
+
+
+def test_mla_tensor_core_single_token_is_exact():
+    q, c, lens = inputs.mla_decode_inputs(11, 2, 32, 512, [1, 20000])
+    assert tc_path(2, 32, [1, 20000]) == 1
+    got = run(q, c, lens)
+    assert torch.equal(got[0], c[0][None].expand(32, -1))
+
+
+def test_mla_tensor_core_nan_in_previous_sequence_stays_there():
+    # sequence 1 (30 tokens) is shorter than a 64-token stage: its box starts inside sequence 0
+    q, c, lens = inputs.mla_decode_inputs(12, 2, 32, 512, [20000, 30])
+    assert tc_path(2, 32, [20000, 30]) == 1
+    c = c.clone()
+    c[19999, 5] = float("nan")
+    got = run(q, c, lens)
+    assert torch.isnan(got[0].float()).any()
+    check(got[1:], oracle.mla_decode(q[1:], c[20000:], lens[1:]), "sequence after a NaN row", v=c[20000:], n_keys=30)
+
+
+def test_mla_tensor_core_running_max_rescale():
+    q, c, lens = spiked_inputs(71, 2, 32, [20000, 300])
+    assert tc_path(2, 32, [20000, 300]) == 1
+    check(run(q, c, lens), oracle.mla_decode(q, c, lens), "MLA with rescales (tensor cores)", v=c, n_keys=20000)

@@ -146,6 +146,16 @@ def test_mla_wait_runs_out(W):
     assert torch.equal(got, gqa.mla_decode(q, c, L))
 
 
+def test_mla_tensor_core_wait_runs_out(W):
+    q, c, L = (t.cuda() for t in inputs.mla_decode_inputs(28, 2, 32, 512, [20000, 300]))
+    assert W.gqa_mla_decode_path(2, 32, 512, c.shape[0]) == 1
+    out = torch.empty_like(q)
+    launch = lambda lib: lib.gqa_mla_decode_rows(q.data_ptr(), c.data_ptr(), c.shape[0], L.data_ptr(),  # noqa: E731
+                                                 out.data_ptr(), 2, 32, 512, 512 ** -0.5, stream())
+    got = stalled_then_clean(W, launch, out)
+    assert torch.equal(got, gqa.mla_decode(q, c, L))
+
+
 def test_product_library_status_clean():
     assert gqa.gqa_get_device_status() == _lib.GQA_OK
 
