@@ -234,3 +234,5 @@ def mla_decode_inputs(seed: int, B: int, h: int, d_c: int, seqlens):
 
 MLA_DECODE = Workload("MLA absorbed decode B16 h32 d_c512 L4096", "decode", 6, B=16, h=32, n_kv=1, d=512,
                       kv_len=4096, notes="latent cache shared by all heads; K = V = c_kv")
+MLA_DECODE_LONG = Workload("MLA absorbed decode B4 h32 d_c512 L65536", "decode", 7, B=4, h=32, n_kv=1, d=512,
+                           kv_len=65536, notes="long sequences in a small batch (the tensor-core kernel's shapes)")

@@ -21,6 +21,7 @@ The same run times, each under its own key:
   decode_fp8, decode_paged, decode_paged_fp8, decode_fp8_mqa
                           the GQA (and MQA) decode workloads over E4M3 and paged caches
   mla_decode              absorbed MLA decode (B=16, h=32, d_c=512, L=4096)
+  mla_decode_long         absorbed MLA decode (B=4, h=32, d_c=512, L=65536; the tcgen05 kernel)
 Under torchrun every rank runs the same per-GPU workload (the (sequence, KV
 head) units are independent: weak scaling, no collective on the data path);
 with --split the decode workload's batch is divided among the ranks instead
@@ -444,13 +445,14 @@ def chunk_prefill_leg(args, device, world):
             "workload": f"chunked prefill B{B} S_q{S_q} past{P} h{h} n_kv{n_kv} d{d}, {ps}-token pages"}
 
 
-def mla_leg(args, device, world):
-    """Absorbed MLA decode, B16 h32 d_c512 L4096 (64 MiB latent cache per step);
-    copies rotated so each step reads a cache L2 has not seen for several steps."""
+def mla_leg(args, device, world, w=None):
+    """Absorbed MLA decode, B16 h32 d_c512 L4096 (64 MiB latent cache per step) unless
+    another MLA workload is given; copies rotated so each step reads a cache L2 has not
+    seen for several steps."""
     import torch
     import attention_gqa_decode_b200 as gqa
     from attention_gqa_decode_b200 import inputs
-    w = inputs.MLA_DECODE
+    w = w or inputs.MLA_DECODE
     q, c, lens = inputs.mla_decode_inputs(w.seed, w.B, w.h, w.d, w.kv_len)
     nbytes = c.numel() * c.element_size()
     copies = max(3, -(-3 * 128 * 1024 * 1024 // nbytes))
@@ -465,7 +467,8 @@ def mla_leg(args, device, world):
     kern_ms = multirank.max_over_ranks(total, device) / steps
     if gqa.gqa_get_device_status() != 0:
         raise RuntimeError("device status after the MLA decode leg")
-    return {"kv_bytes": nbytes, "kernel_ms": kern_ms, "steps": steps, "copies": copies, "workload": w.name}
+    return {"kv_bytes": nbytes, "kernel_ms": kern_ms, "steps": steps, "copies": copies, "workload": w.name,
+            "B": w.B, "path": gqa.gqa_mla_decode_path(w.B, w.h, w.d, int(lens.clamp(min=0).sum()))}
 
 
 def prefill_leg(args, device, world):
@@ -546,6 +549,7 @@ def main():
     pre = None if args.no_prefill else prefill_leg(args, device, world)
     chunk = None if (args.no_prefill or args.no_variants) else chunk_prefill_leg(args, device, world)
     mla = None if args.no_variants else mla_leg(args, device, world)
+    mla_long = None if args.no_variants else mla_leg(args, device, world, inputs.MLA_DECODE_LONG)
     variants = {} if args.no_variants else {
         "decode_fp8": cache_variant_leg("fp8", args, device, world),
         "decode_paged": cache_variant_leg("paged", args, device, world),
@@ -595,15 +599,19 @@ def main():
             "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16"], "unit": "TFLOP/s",
                          "frac": tf / pk["bf16"], "traffic": kernel_traffic("gqa_prefill_kernel[paged]"),
                          "algorithmic_flops_per_launch": chunk["flops"], "peak_source": pk["src"]}}
-    if mla is not None:
-        gbs = mla["kv_bytes"] / (mla["kernel_ms"] / 1e3) / 1e9
-        line["mla_decode"] = {
-            "metric": "MLA decode latent-cache GB/s", "workload": mla["workload"], "value": world * gbs,
-            "unit": "GB/s", "ms_per_call": mla["kernel_ms"], "steps": mla["steps"],
-            "tokens_per_s": world * 16 / (mla["kernel_ms"] / 1e3), "l2": f"{mla['copies']} cache copies rotated",
+    for key, r, tk in (("mla_decode", mla, "gqa_mla_decode_kernel"),
+                       ("mla_decode_long", mla_long, "mla_decode_tc_kernel[long]")):
+        if r is None:
+            continue
+        gbs = r["kv_bytes"] / (r["kernel_ms"] / 1e3) / 1e9
+        line[key] = {
+            "metric": "MLA decode latent-cache GB/s", "workload": r["workload"], "value": world * gbs,
+            "unit": "GB/s", "ms_per_call": r["kernel_ms"], "steps": r["steps"],
+            "kernel": ["warp-level MMA", "tcgen05"][r["path"]],
+            "tokens_per_s": world * r["B"] / (r["kernel_ms"] / 1e3), "l2": f"{r['copies']} cache copies rotated",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
-                         "traffic": kernel_traffic("gqa_mla_decode_kernel"),
-                         "algorithmic_bytes_per_launch": mla["kv_bytes"], "peak_source": pk["src"]}}
+                         "traffic": kernel_traffic(tk),
+                         "algorithmic_bytes_per_launch": r["kv_bytes"], "peak_source": pk["src"]}}
     desc = {"decode_fp8": ("E4M3 cache, one fp32 scale per KV head", "gqa_decode_kernel[e4m3]"),
             "decode_paged": ("bf16 cache in 64-token pages, seeded random page order", "gqa_decode_kernel[paged]"),
             "decode_paged_fp8": ("E4M3 cache in 64-token pages", "gqa_decode_kernel[paged,e4m3]")}
