@@ -14,7 +14,7 @@ _handle = None
 GQA_OK, GQA_ERR_INVALID_ARG, GQA_ERR_UNSUPPORTED, GQA_ERR_CUDA, GQA_ERR_TIMEOUT = range(5)
 
 # every entry point include/gqa.h declares, with its ctypes signature
-_vp, _i, _f, _i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64
+_vp, _i, _f, _i64, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64, ctypes.c_size_t
 SIGNATURES = {
     "gqa_prefill": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_decode": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp], _i),
@@ -29,7 +29,9 @@ SIGNATURES = {
     "gqa_prefill_paged": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _i, _i, _i, _i, _i, _f, _vp], _i),
     "gqa_mla_decode": ([_vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp], _i),
     "gqa_mla_decode_rows": ([_vp, _vp, _i64, _vp, _vp, _i, _i, _i, _f, _vp], _i),
-    "gqa_mla_decode_path": ([_i, _i, _i, _i64], _i),
+    "gqa_mla_decode_path": ([_i, _i, _i, _i64, _i], _i),
+    "gqa_mla_decode_split": ([_vp, _vp, _i64, _vp, _vp, _i, _i, _i, _f, _vp, _sz, _vp], _i),
+    "gqa_mla_decode_split_workspace_bytes": ([_i, _i, _i], _sz),
     "gqa_status_string": ([_i], ctypes.c_char_p),
     "gqa_get_device_status": ([_vp], _i),
 }
@@ -112,8 +114,18 @@ def gqa_mla_decode_rows(q_absorbed, c_kv, cache_rows, seqlens, out, B, h, d_c, s
     return lib().gqa_mla_decode_rows(q_absorbed, c_kv, int(cache_rows), seqlens, out, B, h, d_c, float(scale), stream)
 
 
-def gqa_mla_decode_path(B, h, d_c, cache_rows) -> int:
-    return lib().gqa_mla_decode_path(B, h, d_c, int(cache_rows))
+def gqa_mla_decode_path(B, h, d_c, cache_rows, with_workspace=0) -> int:
+    return lib().gqa_mla_decode_path(B, h, d_c, int(cache_rows), int(with_workspace))
+
+
+def gqa_mla_decode_split(q_absorbed, c_kv, cache_rows, seqlens, out, B, h, d_c, scale, workspace, workspace_bytes,
+                         stream) -> int:
+    return lib().gqa_mla_decode_split(q_absorbed, c_kv, int(cache_rows), seqlens, out, B, h, d_c, float(scale),
+                                      workspace, workspace_bytes, stream)
+
+
+def gqa_mla_decode_split_workspace_bytes(B, h, d_c) -> int:
+    return lib().gqa_mla_decode_split_workspace_bytes(B, h, d_c)
 
 
 def gqa_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, B, h, n_kv, d_h, scale, stream) -> int:
@@ -466,10 +478,12 @@ def prefill_paged(q, k_new, v_new, k_pages, v_pages, block_table, past_lens, sca
     return out
 
 
-def mla_decode(q_absorbed, c_kv, seqlens, scale: float | None = None, out=None, stream=None):
+def mla_decode(q_absorbed, c_kv, seqlens, scale: float | None = None, out=None, stream=None, workspace=None):
     """Absorbed MLA decode: q_absorbed [B,h,d_c], packed latent cache c_kv [sum(seqlens),d_c] (bf16,
     CUDA), seqlens int32 [B].  Returns softmax(q' c^T * scale) c as bf16 [B,h,d_c];
-    ``scale=None`` is d_c ** -0.5."""
+    ``scale=None`` is d_c ** -0.5.  Shapes for which gqa_mla_decode_path(..., 1) is 2
+    run through gqa_mla_decode_split with ``workspace`` (default: the binding's
+    per-device workspace, :func:`split_workspace`); the rest through gqa_mla_decode_rows."""
     import torch
     _check(q_absorbed, "q_absorbed", 3), _check(c_kv, "c_kv", 2)
     B, h, d_c = q_absorbed.shape
@@ -485,8 +499,17 @@ def mla_decode(q_absorbed, c_kv, seqlens, scale: float | None = None, out=None, 
         if out.shape != q_absorbed.shape:
             raise ValueError("out must have q_absorbed's shape")
     with torch.cuda.device(q_absorbed.device):
-        st = gqa_mla_decode_rows(q_absorbed.data_ptr(), c_kv.data_ptr(), c_kv.shape[0], seqlens.data_ptr(),
-                                 out.data_ptr(), B, h, d_c, scale, _stream_ptr(stream))
+        if gqa_mla_decode_path(B, h, d_c, c_kv.shape[0], 1) == 2:
+            need = gqa_mla_decode_split_workspace_bytes(B, h, d_c)
+            ws = workspace if workspace is not None else split_workspace(q_absorbed.device, need)
+            st = gqa_mla_decode_split(q_absorbed.data_ptr(), c_kv.data_ptr(), c_kv.shape[0], seqlens.data_ptr(),
+                                      out.data_ptr(), B, h, d_c, scale, ws.data_ptr(), ws.numel() * ws.element_size(),
+                                      _stream_ptr(stream))
+            where = "gqa_mla_decode_split"
+        else:
+            st = gqa_mla_decode_rows(q_absorbed.data_ptr(), c_kv.data_ptr(), c_kv.shape[0], seqlens.data_ptr(),
+                                     out.data_ptr(), B, h, d_c, scale, _stream_ptr(stream))
+            where = "gqa_mla_decode_rows"
     if st != GQA_OK:
-        raise GQAError(st, "gqa_mla_decode_rows")
+        raise GQAError(st, where)
     return out

@@ -29,6 +29,10 @@ int launch_prefill_paged(const void *q, const void *k_new, const void *v_new, vo
 int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h, float scale,
                       long long cache_rows, bool rows_known, cudaStream_t stream);
 bool mla_prefers_tc(int B, int h, long long cache_rows, bool rows_known, int sms);
+bool mla_ws_prefers_tc(int B, int h, long long cache_rows, int sms);
+size_t mla_ws_bytes(int B, int h, int sms);
+int launch_mla_decode_ws(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h,
+                         float scale, long long cache_rows, void *ws, size_t ws_bytes, cudaStream_t stream);
 int launch_decode_ex(const void *q, const void *k, const void *v, const float *k_scale, const float *v_scale,
                      const int32_t *seqlens, const int32_t *block_table, int max_blocks, int page_size,
                      int num_pages, void *out, int B, int h, int n_kv, int d, float scale, long long cache_rows,
@@ -332,9 +336,34 @@ int gqa_mla_decode_rows(const void *q_absorbed, const void *c_kv, int64_t cache_
     return mla_decode(q_absorbed, c_kv, cache_rows, true, seqlens, out, B, h, d_c, scale, stream);
 }
 
-int gqa_mla_decode_path(int B, int h, int d_c, int64_t cache_rows) {
+int gqa_mla_decode_path(int B, int h, int d_c, int64_t cache_rows, int with_workspace) {
     if (B <= 0 || h <= 0 || d_c != 512 || !rows_ok(cache_rows)) return -1;
-    return gqa::mla_prefers_tc(B, h, cache_rows, true, gqa_host::sm_count()) ? 1 : 0;
+    const int sms = gqa_host::sm_count();
+    if (with_workspace && gqa::mla_ws_prefers_tc(B, h, cache_rows, sms)) return 2;
+    return gqa::mla_prefers_tc(B, h, cache_rows, true, sms) ? 1 : 0;
+}
+
+static bool mla_sizes_ok(int B, int h) { return B > 0 && B <= 65535 && h > 0 && h <= 65535 * 16; }
+
+size_t gqa_mla_decode_split_workspace_bytes(int B, int h, int d_c) {
+    if (!mla_sizes_ok(B, h) || d_c != 512) return 0;
+    return gqa::mla_ws_bytes(B, h, gqa_host::sm_count());
+}
+
+int gqa_mla_decode_split(const void *q_absorbed, const void *c_kv, int64_t cache_rows, const int32_t *seqlens,
+                         void *out, int B, int h, int d_c, float scale, void *workspace, size_t workspace_bytes,
+                         cudaStream_t stream) {
+    if (!rows_ok(cache_rows)) return GQA_ERR_INVALID_ARG;
+    if (!q_absorbed || !c_kv || !seqlens || !out || !workspace) return GQA_ERR_INVALID_ARG;
+    if (!aligned16(q_absorbed) || !aligned16(c_kv) || !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return GQA_ERR_INVALID_ARG;
+    if (!mla_sizes_ok(B, h)) return GQA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return GQA_ERR_INVALID_ARG;
+    if (d_c != 512) return GQA_ERR_UNSUPPORTED;
+    const int st = gqa::launch_mla_decode_ws(q_absorbed, c_kv, seqlens, out, B, h, scale, cache_rows, workspace,
+                                             workspace_bytes, stream);
+    return st == 0 ? GQA_OK : st == 1 ? GQA_ERR_INVALID_ARG : GQA_ERR_CUDA;
 }
 
 const char *gqa_status_string(int status) {

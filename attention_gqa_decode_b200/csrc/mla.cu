@@ -471,7 +471,8 @@ __global__ void __launch_bounds__(kMlaThreads, 2)
 // host launcher
 
 int launch_mla_decode_tc(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h,
-                         float scale, long long cache_rows, cudaStream_t stream);
+                         float scale, long long cache_rows, void *ws, size_t ws_bytes, cudaStream_t stream);
+size_t mla_tc_workspace_bytes(int B, int h, int sms);
 
 // The tensor-core kernel (mla_tc.cu) for long sequences in batches too small to
 // fill the GPU with this kernel: more than 16 heads (its products are 32 heads
@@ -482,17 +483,38 @@ int launch_mla_decode_tc(const void *q, const void *c_kv, const int32_t *seqlens
 // fills the SMs (B16 h32 L4096 34 / 46) or on short or 16-head work.
 constexpr long long kMlaTcMinAvgRows = 8192;
 
+// This kernel's CTAs for a shape: 16-head groups x sequences, each in up to 8 splits (two
+// CTAs per SM).
+static long mla_warp_level_ctas(int B, int h, int sms) {
+    const long units = static_cast<long>(B) * ((h + kMlaHeads - 1) / kMlaHeads);
+    return units * std::max(1L, std::min(static_cast<long>(kMlaMaxSplit), 2L * sms / units));
+}
+
 bool mla_prefers_tc(int B, int h, long long cache_rows, bool rows_known, int sms) {
     if (!rows_known || h <= kMlaHeads) return false;
-    const long units = static_cast<long>(B) * ((h + kMlaHeads - 1) / kMlaHeads);
-    const long P = std::max(1L, std::min(static_cast<long>(kMlaMaxSplit), 2L * sms / units));
-    return units * P < sms && cache_rows >= kMlaTcMinAvgRows * B;
+    return mla_warp_level_ctas(B, h, sms) < sms && cache_rows >= kMlaTcMinAvgRows * B;
 }
+
+// With a workspace the tensor-core kernel's splits merge there instead of in a cluster, so
+// it keeps every SM busy (one CTA per SM, any number of splits): taken in the same regime
+// (h > 16, this kernel's CTAs fewer than the SMs) down to kMlaWsMinAvgRows tokens per
+// sequence.  Measured on B200 (us, this kernel / tensor cores with the workspace):
+// B8 h32 L8192 57.9 / 37.7, B2 h32 L8192 47.7 / 21.8, B4 h32 L65536 340.5 / 108.3,
+// B1 h32 L20000 108.7 / 28.9; where this kernel fills the SMs it stays ahead
+// (B16 h32 L4096 34.3 / 37.7, B16 h64 L4096 58.7 / 61.5, B32 h32 L2048 34.1 / 37.8).
+constexpr long long kMlaWsMinAvgRows = 2048;
+
+bool mla_ws_prefers_tc(int B, int h, long long cache_rows, int sms) {
+    if (h <= kMlaHeads) return false;
+    return mla_warp_level_ctas(B, h, sms) < sms && cache_rows >= kMlaWsMinAvgRows * B;
+}
+
+size_t mla_ws_bytes(int B, int h, int sms) { return mla_tc_workspace_bytes(B, h, sms); }
 
 int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h, float scale,
                       long long cache_rows, bool rows_known, cudaStream_t stream) {
     if (mla_prefers_tc(B, h, cache_rows, rows_known, gqa_host::sm_count()))
-        return launch_mla_decode_tc(q, c_kv, seqlens, out, B, h, scale, cache_rows, stream);
+        return launch_mla_decode_tc(q, c_kv, seqlens, out, B, h, scale, cache_rows, nullptr, 0, stream);
     auto kern = gqa_mla_decode_kernel;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 3;
@@ -539,6 +561,16 @@ int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, v
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, tc, prm) != cudaSuccess) return 3;
     return 0;
+}
+
+// 0 = launched, 1 = workspace too small, 3 = a CUDA call failed.
+int launch_mla_decode_ws(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h,
+                         float scale, long long cache_rows, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    const int sms = gqa_host::sm_count();
+    if (ws_bytes < mla_ws_bytes(B, h, sms)) return 1;
+    if (mla_ws_prefers_tc(B, h, cache_rows, sms))
+        return launch_mla_decode_tc(q, c_kv, seqlens, out, B, h, scale, cache_rows, ws, ws_bytes, stream);
+    return launch_mla_decode(q, c_kv, seqlens, out, B, h, scale, cache_rows, true, stream);
 }
 
 }  // namespace gqa

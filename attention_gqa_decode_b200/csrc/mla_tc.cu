@@ -62,7 +62,9 @@ constexpr int kPairBytes = 2 * kPanelBytes;             // 128 dims: one M block
 constexpr int kPairs = kDc / 128;                       // pairs per stage
 constexpr int kSlots = 12;                              // ring of pair slots (three stages)
 constexpr int kThreads = 6 * 32;                        // 0 softmax, 0-3 O^T lanes, 4 TMA, 5 MMA
-constexpr int kMaxSplit = 16;
+constexpr int kMaxSplit = 16;                          // splits of one cluster (its largest size)
+constexpr int kMaxSplitWs = 256;                        // splits merged through a workspace
+constexpr int kPartFloats = kHeads * kDc + 2 * kHeads;  // a workspace partial: O [32][512], m [32], l [32]
 constexpr float kRescale = 8.0f;                        // lazy rescale threshold (log2 units)
 constexpr int kSplitAllBelow = 256;                     // remainder product for sequences this short
 // TMEM columns
@@ -78,6 +80,7 @@ struct Params {
     long long cache_rows;          // rows the latent cache holds (the tensor map's extent)
     float scale_log2;              // scale * log2(e), >= 0
     int *status;
+    float *part;                   // null: the splits merge in their cluster; else [CTA][kPartFloats]
     GQA_TEST_STALL_FIELD
 };
 
@@ -129,6 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int grp = blockIdx.y, b = blockIdx.z;
     const int head0 = grp * kHeads;
     const int HS = min(p.h - head0, kHeads);
+    // with a workspace, the merge launch that follows may start now (it waits for this grid)
+    if (p.part) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kSlots; ++i) {
@@ -504,10 +509,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();   // every role has finished; the producer has drained its copies
     tc_fence_after();
+    const bool good = (*abort_flag == 0);
+    if (p.part) {
+        // this split's partial into the workspace (unnormalised O, running max, sum), read by
+        // the merge launch; rows past the group are left unwritten
+        float *pp = p.part + static_cast<size_t>((b * gridDim.y + grp) * P + split) * kPartFloats;
+        if (warp < 4 && good) {
+            const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+#pragma unroll 1
+            for (int j = 0; j < kPairs; ++j) {
+                uint32_t o[32];
+                if (n_stages > 0) {
+                    tmem_ld32(tmem + kColO + 32 * j + lane_off, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = 0u;
+                }
+                const int d = 128 * j + 32 * warp + lane;
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if (e < HS) pp[e * kDc + d] = __uint_as_float(o[e]);
+            }
+            if (warp == 0 && lane < HS) {
+                pp[kHeads * kDc + lane] = n_stages > 0 ? m_run : -INFINITY;
+                pp[kHeads * kDc + kHeads + lane] = l_run;
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 5) {
+            tc_fence_after();
+            tmem_dealloc(tmem, 512);
+        }
+        return;
+    }
     float *co = reinterpret_cast<float *>(sRing);              // [32 heads][512] fp32
     float *cm = reinterpret_cast<float *>(sRing + SM::kOffCm);  // [32]
     float *cl = cm + 32;                                        // [32]
-    const bool good = (*abort_flag == 0);
     if (warp < 4 && good) {
         const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
 #pragma unroll 1
@@ -606,6 +645,72 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster.sync();
 }
 
+// The merge of the workspace partials: one block per (sequence x group, head), eight warps
+// each folding every eighth split with the log-sum-exp rule (running max, sum, unnormalised
+// O; a lane holds 16 of the 512 dims), then the eight folds combined through shared memory.
+constexpr int kMergeWarps = 8;
+
+__global__ void __launch_bounds__(kMergeWarps * 32)
+    mla_merge_kernel(const float *part, __nv_bfloat16 *out, int h, int groups, int P) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // the partials' launch has completed
+    __shared__ float sM[kMergeWarps], sL[kMergeWarps];
+    __shared__ float4 sO[kMergeWarps][kDc / 4];
+    const int u = blockIdx.x, r = blockIdx.y;
+    const int grp = u % groups, b = u / groups;
+    const int head = grp * kHeads + r;
+    if (head >= h) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float M = -INFINITY, L = 0.f;
+    float4 acc[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+    for (int q = warp; q < P; q += kMergeWarps) {
+        const float *pp = part + static_cast<size_t>(u * P + q) * kPartFloats;
+        const float m = __ldcg(pp + kHeads * kDc + r);
+        const float l = __ldcg(pp + kHeads * kDc + kHeads + r);
+        float4 o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o[k] = __ldcg(reinterpret_cast<const float4 *>(pp + r * kDc) + lane + 32 * k);
+        if (m == -INFINITY) continue;   // a split with no tokens
+        const float M2 = fmaxf(M, m);
+        const float a = exp2f(M - M2), w = exp2f(m - M2);   // M2 is finite: a = 0 while M is -inf
+        L = L * a + l * w;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            acc[k] = make_float4(acc[k].x * a + o[k].x * w, acc[k].y * a + o[k].y * w, acc[k].z * a + o[k].z * w,
+                                 acc[k].w * a + o[k].w * w);
+        M = M2;
+    }
+    if (lane == 0) {
+        sM[warp] = M;
+        sL[warp] = L;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) sO[warp][lane + 32 * k] = acc[k];
+    __syncthreads();
+    float Mf = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) Mf = fmaxf(Mf, sM[w]);
+    float wt[kMergeWarps], Lf = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) {
+        wt[w] = sM[w] == -INFINITY ? 0.f : exp2f(sM[w] - Mf);
+        Lf += wt[w] * sL[w];
+    }
+    const float inv = Lf > 0.f ? 1.f / Lf : 0.f;
+    // thread t writes dims 2t, 2t + 1
+    const float *so = reinterpret_cast<const float *>(sO);
+    float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) {
+        x0 += wt[w] * so[w * kDc + 2 * threadIdx.x];
+        x1 += wt[w] * so[w * kDc + 2 * threadIdx.x + 1];
+    }
+    *reinterpret_cast<__nv_bfloat162 *>(out + (static_cast<size_t>(b) * h + head) * kDc + 2 * threadIdx.x) =
+        __floats2bfloat162_rn(x0 * inv, x1 * inv);
+}
+
 }  // namespace mla_tc
 
 // ---------------------------------------------------------------------------
@@ -644,8 +749,22 @@ int max_active_clusters_tc(int P) {
 
 }  // namespace
 
+// Splits per (sequence, 32-head group) when they merge through a workspace: one CTA per SM.
+static int mla_tc_ws_splits(long units, int sms) {
+    return static_cast<int>(std::max(1L, std::min(static_cast<long>(mla_tc::kMaxSplitWs), sms / units)));
+}
+
+size_t mla_tc_workspace_bytes(int B, int h, int sms) {
+    const long units = static_cast<long>(B) * ((h + mla_tc::kHeads - 1) / mla_tc::kHeads);
+    return static_cast<size_t>(units) * mla_tc_ws_splits(units, sms) * mla_tc::kPartFloats * sizeof(float);
+}
+
+// ws == null: the splits of a sequence form a cluster (at most 16, as many as fit at once) and
+// merge in it.  Otherwise one CTA per SM (any number of splits) writes its partial to ws, and
+// a second launch merges them (programmatic dependent launch: it is scheduled while the
+// first runs and waits for it).  0 = launched, 1 = ws too small, 3 = a CUDA call failed.
 int launch_mla_decode_tc(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h,
-                         float scale, long long cache_rows, cudaStream_t stream) {
+                         float scale, long long cache_rows, void *ws, size_t ws_bytes, cudaStream_t stream) {
     using namespace mla_tc;
     auto kern = mla_decode_tc_kernel;
     int dev = 0;
@@ -657,6 +776,8 @@ int launch_mla_decode_tc(const void *q, const void *c_kv, const int32_t *seqlens
                    cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
         }))
         return 3;
+    const int sms = gqa_host::sm_count();
+    if (ws && ws_bytes < mla_tc_workspace_bytes(B, h, sms)) return 1;
     CUtensorMap tc;
     // token extent = the cache's rows (the kernel cuts lengths that ask for more and reports them)
     const uint64_t dims[2] = {static_cast<uint64_t>(kDc), static_cast<uint64_t>(std::max(cache_rows, 1LL))};
@@ -666,9 +787,13 @@ int launch_mla_decode_tc(const void *q, const void *c_kv, const int32_t *seqlens
 
     const int groups = (h + kHeads - 1) / kHeads;
     const long units = static_cast<long>(B) * groups;
-    // one CTA per SM: the most splits whose clusters all fit at once
-    int P = static_cast<int>(std::max(1L, std::min(static_cast<long>(kMaxSplit), gqa_host::sm_count() / units)));
-    while (P > 1 && max_active_clusters_tc(P) < units) --P;
+    int P;
+    if (ws) {
+        P = mla_tc_ws_splits(units, sms);
+    } else {   // one CTA per SM: the most splits whose clusters all fit at once
+        P = static_cast<int>(std::max(1L, std::min(static_cast<long>(kMaxSplit), sms / units)));
+        while (P > 1 && max_active_clusters_tc(P) < units) --P;
+    }
     Params prm;
     prm.q = static_cast<const __nv_bfloat16 *>(q);
     prm.seqlens = seqlens;
@@ -679,6 +804,7 @@ int launch_mla_decode_tc(const void *q, const void *c_kv, const int32_t *seqlens
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.status = gqa_host::device_status();
     if (!prm.status) return 3;
+    prm.part = static_cast<float *>(ws);
     GQA_SET_TEST_STALL(prm);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(P, groups, B);
@@ -687,12 +813,30 @@ int launch_mla_decode_tc(const void *q, const void *c_kv, const int32_t *seqlens
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = P;
+    attr[0].val.clusterDim.x = ws ? 1 : P;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, kern, tc, prm) != cudaSuccess) return 3;
+    if (!ws) return 0;
+    // the merge: one block per (sequence x group, head)
+    cudaLaunchConfig_t mc = {};
+    mc.gridDim = dim3(static_cast<unsigned>(units), kHeads, 1);
+    mc.blockDim = dim3(kMergeWarps * 32, 1, 1);
+    mc.stream = stream;
+    cudaLaunchAttribute ma[1];
+    ma[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    ma[0].val.programmaticStreamSerializationAllowed = 1;
+    mc.attrs = ma;
+    mc.numAttrs = 1;
+    const float *cpart = static_cast<const float *>(ws);
+    __nv_bfloat16 *cout = static_cast<__nv_bfloat16 *>(out);
+    if (cudaLaunchKernelEx(&mc, mla_merge_kernel, cpart, cout, h, groups, P) != cudaSuccess) {
+        cudaGetLastError();   // without programmatic launch (stream order still holds)
+        mla_merge_kernel<<<mc.gridDim, mc.blockDim, 0, stream>>>(cpart, cout, h, groups, P);
+        if (cudaGetLastError() != cudaSuccess) return 3;
+    }
     return 0;
 }
 

@@ -319,15 +319,48 @@ int gqa_mla_decode_rows(const void *q_absorbed, const void *c_kv, int64_t cache_
                         const int32_t *seqlens, void *out,
                         int B, int h, int d_c, float scale, cudaStream_t stream);
 
-/* Which kernel gqa_mla_decode_rows runs for a shape on the current device:
- * 0 = warp-level MMA (16-head groups, splits of one sequence merged in a
- * thread-block cluster; gqa_mla_decode always runs it), 1 = 5th-generation
- * tensor cores (32-head groups, q' resident in tensor memory, one CTA per SM),
- * taken when h > 16, the warp-level kernel's CTAs (B * ceil(h / 16) times up
- * to 8 splits) are fewer than the SMs, and cache_rows >= 8192 * B.  Host-only
- * (reads the SM count; 148 when no device answers).  Returns -1 for B <= 0,
- * h <= 0, d_c != 512 or cache_rows outside [0, 2^31). */
-int gqa_mla_decode_path(int B, int h, int d_c, int64_t cache_rows);
+/*
+ * gqa_mla_decode_rows with a workspace: the tensor-core kernel can then split a
+ * sequence over any number of SMs (one CTA per SM) and merge the splits' partial
+ * results from the workspace in a second launch (log-sum-exp rule), instead of
+ * within a thread-block cluster of at most 16.  Used where gqa_mla_decode_path
+ * (..., 1) answers 2; otherwise the call runs as gqa_mla_decode_rows and the
+ * workspace is not touched.
+ *   workspace        DEVICE memory of at least
+ *                    gqa_mla_decode_split_workspace_bytes(B, h, d_c) bytes,
+ *                    256-byte aligned, owned by the caller, needing no
+ *                    initialisation.  Calls that share a workspace must not
+ *                    overlap on the GPU.
+ * Errors: as gqa_mla_decode_rows, plus GQA_ERR_INVALID_ARG for a null,
+ * misaligned or too small workspace.
+ */
+int gqa_mla_decode_split(const void *q_absorbed, const void *c_kv, int64_t cache_rows,
+                         const int32_t *seqlens, void *out,
+                         int B, int h, int d_c, float scale,
+                         void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Bytes of workspace gqa_mla_decode_split needs on the current device (the
+ * tensor-core kernel's partials: ceil(h / 32) * B * splits * (32 * 512 + 64)
+ * floats, with splits = max(1, min(256, SMs / (ceil(h / 32) * B)))); 0 for
+ * sizes it refuses (B <= 0 or > 65535, h <= 0 or > 65535 * 16, d_c != 512).
+ * Host-only. */
+size_t gqa_mla_decode_split_workspace_bytes(int B, int h, int d_c);
+
+/* Which kernel runs for a shape on the current device: gqa_mla_decode_rows
+ * (with_workspace = 0) or gqa_mla_decode_split (with_workspace != 0).
+ *   0  warp-level MMA: 16-head groups, the splits of one sequence merged in a
+ *      thread-block cluster (gqa_mla_decode always runs it);
+ *   1  5th-generation tensor cores with q' resident in tensor memory, 32-head
+ *      groups, one CTA per SM, splits merged in a cluster: taken when h > 16,
+ *      the warp-level kernel's CTAs (B * ceil(h / 16) times up to 8 splits) are
+ *      fewer than the SMs, and cache_rows >= 8192 * B;
+ *   2  the same tensor-core kernel with its splits merged through the workspace
+ *      (with_workspace only; any number of splits, every SM busy): taken when
+ *      h > 16, the warp-level kernel's CTAs are fewer than the SMs, and
+ *      cache_rows >= 2048 * B.
+ * Host-only (reads the SM count; 148 when no device answers).  Returns -1 for
+ * B <= 0, h <= 0, d_c != 512 or cache_rows outside [0, 2^31). */
+int gqa_mla_decode_path(int B, int h, int d_c, int64_t cache_rows, int with_workspace);
 
 /* A static, human-readable name for a gqa_status_t value. */
 const char *gqa_status_string(int status);

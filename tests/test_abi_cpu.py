@@ -222,17 +222,32 @@ def test_split_workspace_bytes_is_zero_for_rejected_sizes(L, B, h, n_kv, d):
     assert L.gqa_decode_split_workspace_bytes(B, h, n_kv, d) == 0
 
 
-@pytest.mark.parametrize("B,h,d_c,rows,want", [
-    (16, 32, 512, 16 * 4096, 0),    # the warp-level kernel fills the SMs (32 groups x 8 splits)
-    (8, 32, 512, 8 * 32768, 1),     # 128 warp-level CTAs, long sequences
-    (1, 32, 512, 20000, 1),
-    (1, 32, 512, 8191, 0),          # under 8192 rows per sequence
-    (1, 16, 512, 100000, 0),        # 16 heads: one warp-level group is as wide
-    (4, 64, 512, 4 * 16384, 1),
-    (5, 64, 512, 5 * 16384, 0),     # 20 groups x 8 splits = 160 CTAs
-    (0, 32, 512, 0, -1), (1, 0, 512, 10, -1), (1, 32, 256, 10, -1), (1, 32, 512, -1, -1), (1, 32, 512, 2 ** 31, -1),
+@pytest.mark.parametrize("B,h,d_c,rows,want,want_ws", [
+    (16, 32, 512, 16 * 4096, 0, 0),    # the warp-level kernel fills the SMs (32 groups x 8 splits)
+    (8, 32, 512, 8 * 32768, 1, 2),     # 128 warp-level CTAs, long sequences
+    (1, 32, 512, 20000, 1, 2),
+    (1, 32, 512, 8191, 0, 2),          # under 8192 rows per sequence (2048 with a workspace)
+    (1, 32, 512, 2047, 0, 0),
+    (1, 16, 512, 100000, 0, 0),        # 16 heads: one warp-level group is as wide
+    (4, 64, 512, 4 * 16384, 1, 2),
+    (5, 64, 512, 5 * 16384, 0, 0),     # 20 groups x 8 splits = 160 warp-level CTAs
+    (8, 32, 512, 8 * 2048, 0, 2),      # 2048 rows per sequence are enough with a workspace
+    (0, 32, 512, 0, -1, -1), (1, 0, 512, 10, -1, -1), (1, 32, 256, 10, -1, -1), (1, 32, 512, -1, -1, -1),
+    (1, 32, 512, 2 ** 31, -1, -1),
 ], ids=str)
-def test_mla_decode_path_rule(L, B, h, d_c, rows, want):
-    """gqa_mla_decode_path: the shape rule between the warp-level and the tensor-core MLA
-    kernels as gqa.h states it, at the 148 SMs a B200 has (and the count assumed without one)."""
-    assert L.gqa_mla_decode_path(B, h, d_c, rows) == want
+def test_mla_decode_path_rule(L, B, h, d_c, rows, want, want_ws):
+    """gqa_mla_decode_path: the shape rules between the warp-level and the tensor-core MLA
+    kernels as gqa.h states them, at the 148 SMs a B200 has (and the count assumed without one)."""
+    assert L.gqa_mla_decode_path(B, h, d_c, rows, 0) == want
+    assert L.gqa_mla_decode_path(B, h, d_c, rows, 1) == want_ws
+
+
+@pytest.mark.parametrize("B,h,d_c,want", [
+    (16, 32, 512, 16 * 9 * 65792),     # nine splits per sequence
+    (1, 32, 512, 148 * 65792),         # one sequence over every SM
+    (300, 32, 512, 300 * 65792),       # one split each
+    (2, 80, 512, 6 * 24 * 65792),      # three 32-head groups
+    (0, 32, 512, 0), (70000, 32, 512, 0), (1, 0, 512, 0), (1, 32, 256, 0),
+], ids=str)
+def test_mla_split_workspace_bytes(L, B, h, d_c, want):
+    assert L.gqa_mla_decode_split_workspace_bytes(B, h, d_c) == want

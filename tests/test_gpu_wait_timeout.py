@@ -148,10 +148,27 @@ def test_mla_wait_runs_out(W):
 
 def test_mla_tensor_core_wait_runs_out(W):
     q, c, L = (t.cuda() for t in inputs.mla_decode_inputs(28, 2, 32, 512, [20000, 300]))
-    assert W.gqa_mla_decode_path(2, 32, 512, c.shape[0]) == 1
+    assert W.gqa_mla_decode_path(2, 32, 512, c.shape[0], 0) == 1
     out = torch.empty_like(q)
     launch = lambda lib: lib.gqa_mla_decode_rows(q.data_ptr(), c.data_ptr(), c.shape[0], L.data_ptr(),  # noqa: E731
                                                  out.data_ptr(), 2, 32, 512, 512 ** -0.5, stream())
+    got = stalled_then_clean(W, launch, out)
+    want = torch.empty_like(q)   # the product library through the same entry (mla_decode takes the workspace path)
+    assert gqa.gqa_mla_decode_rows(q.data_ptr(), c.data_ptr(), c.shape[0], L.data_ptr(), want.data_ptr(), 2, 32, 512,
+                                   512 ** -0.5, stream()) == _lib.GQA_OK
+    torch.cuda.synchronize()
+    assert torch.equal(got, want)
+
+
+def test_mla_tensor_core_workspace_wait_runs_out(W):
+    q, c, L = (t.cuda() for t in inputs.mla_decode_inputs(29, 2, 32, 512, [20000, 300]))
+    assert W.gqa_mla_decode_path(2, 32, 512, c.shape[0], 1) == 2
+    nbytes = W.gqa_mla_decode_split_workspace_bytes(2, 32, 512)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    launch = lambda lib: lib.gqa_mla_decode_split(q.data_ptr(), c.data_ptr(), c.shape[0], L.data_ptr(),  # noqa: E731
+                                                  out.data_ptr(), 2, 32, 512, 512 ** -0.5, ws.data_ptr(), nbytes,
+                                                  stream())
     got = stalled_then_clean(W, launch, out)
     assert torch.equal(got, gqa.mla_decode(q, c, L))
 
