@@ -42,18 +42,6 @@ namespace gqa {
 
 namespace mla_tc {
 
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 constexpr int kDc = 512;                                // latent width
 constexpr int kTok = 64;                                // tokens per stage (N of the score MMA)
 constexpr int kHeads = 32;                              // heads per CTA (N of the P V MMA)
@@ -61,7 +49,7 @@ constexpr int kPanelBytes = kTok * 128;                 // 64 tokens x 64 dims
 constexpr int kPairBytes = 2 * kPanelBytes;             // 128 dims: one M block of O^T
 constexpr int kPairs = kDc / 128;                       // pairs per stage
 constexpr int kSlots = 12;                              // ring of pair slots (three stages)
-constexpr int kThreads = 6 * 32;                        // 0 softmax, 0-3 O^T lanes, 4 TMA, 5 MMA
+constexpr int kThreads = 7 * 32;                        // 0 softmax, 0-3 O^T lanes, 4 TMA, 5 S MMAs, 6 O^T MMAs
 constexpr int kMaxSplit = 16;                          // splits of one cluster (its largest size)
 constexpr int kMaxSplitWs = 256;                        // splits merged through a workspace
 constexpr int kPartFloats = kHeads * kDc + 2 * kHeads;  // a workspace partial: O [32][512], m [32], l [32]
@@ -120,10 +108,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *pvdone = pfull + 2;                          // [2] the stage's P V products completed
     uint64_t *ack = pvdone + 2;                            // [2] warps 1-3 read the decision (and rescaled)
     uint64_t *odone = ack + 2;
-    uint64_t *drain = odone + 1;
+    uint64_t *drain = odone + 1;                           // the S issuer's products completed
+    uint64_t *drain_o = drain + 1;                         // the O^T issuer's, when it gave up
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(ctrl + 320);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 324);
-    long long *red = reinterpret_cast<long long *>(ctrl + 328);          // [6]
+    long long *red = reinterpret_cast<long long *>(ctrl + 328);          // [7]
     float *av = reinterpret_cast<float *>(ctrl + 384);                   // [2][32] rescale factor per head
     volatile int *rflag = reinterpret_cast<volatile int *>(ctrl + 640);  // [2] the stage rescales O^T
 
@@ -151,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(odone, 1);
         mbar_init(drain, 1);
+        mbar_init(drain_o, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -218,91 +208,72 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 5) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 5 || warp == 6) {
+        // ------------------------------------------------------------ MMA issuers: S (warp 5), O^T (warp 6)
+        // Two issuing threads, each committing only its own products, so that neither waits on
+        // the other's condition: O^T(i) issues as soon as its weights are written, whether or
+        // not the stage after it has landed.
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTok, false, false);
             constexpr uint32_t idesc_o = idesc_bf16_f32(128, kHeads, true, false);
             const uint32_t ring_base = smem_u32(sRing);
             const uint32_t p_base = smem_u32(sP);
             auto slot_addr = [&](int i, int j) { return ring_base + ((i * kPairs + j) % kSlots) * kPairBytes; };
-            auto issue_s = [&](int i) {
-                const uint32_t tS = tmem + kColS + (i & 1) * kTok;
+            if (warp == 5) {
+                ok = mbar_wait(qready, 0, abort_flag, p.status);
+                for (int i = 0; i < n_stages && ok; ++i) {
+                    // S(i) reuses the buffer of S(i - 2): after the softmax read it
+                    if (i >= 2 && !mbar_wait(&sfree[i & 1], ((i - 2) >> 1) & 1, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    for (int j = 0; j < kPairs && ok; ++j) {
+                        const int n = i * kPairs + j;
+                        ok = mbar_wait(&full[n % kSlots], (n / kSlots) & 1, abort_flag, p.status);
+                    }
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t tS = tmem + kColS + (i & 1) * kTok;
 #pragma unroll
-                for (int ks = 0; ks < kDc / 16; ++ks) {
-                    // k-step ks: pair ks / 8, panel (ks / 4) % 2, 32-byte column (ks % 4) of the 128-byte rows
-                    const uint32_t bad = slot_addr(i, ks >> 3) + ((ks >> 2) & 1) * kPanelBytes + (ks & 3) * 32;
-                    umma_ts(tS, tmem + kColQ + ks * 8, sdesc_sw128(bad, 16, 1024), idesc_s, ks ? 1u : 0u);
+                    for (int ks = 0; ks < kDc / 16; ++ks) {
+                        // k-step ks: pair ks / 8, panel (ks / 4) % 2, 32-byte column (ks % 4) of the 128-byte rows
+                        const uint32_t bad = slot_addr(i, ks >> 3) + ((ks >> 2) & 1) * kPanelBytes + (ks & 3) * 32;
+                        umma_ts(tS, tmem + kColQ + ks * 8, sdesc_sw128(bad, 16, 1024), idesc_s, ks ? 1u : 0u);
+                    }
+                    umma_commit(&sfull[i & 1]);
                 }
-                umma_commit(&sfull[i & 1]);
-            };
-            auto issue_o = [&](int i) {
-                const uint32_t pb = p_base + (i & 1) * 2 * Smem::kPT;
-                // block by block, each slot released as soon as its products complete
+                umma_commit(drain);   // every S product complete before TMEM is freed
+                mbar_wait_drain(drain, 0, p.status);
+            } else {
+                for (int i = 0; i < n_stages && ok; ++i) {
+                    if (!mbar_wait(&pfull[i & 1], (i >> 1) & 1, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t pb = p_base + (i & 1) * 2 * Smem::kPT;
+                    // block by block, each slot released as soon as its products complete
 #pragma unroll
-                for (int j = 0; j < kPairs; ++j) {
-#pragma unroll
-                    for (int kk = 0; kk < kTok / 16; ++kk)
-                        umma_ss(tmem + kColO + 32 * j, sdesc_sw128(slot_addr(i, j) + kk * 16 * 128, kPanelBytes, 1024),
-                                sdesc_sw128(pb + kk * 32, 16, 1024), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-                    if (rem) {
+                    for (int j = 0; j < kPairs; ++j) {
 #pragma unroll
                         for (int kk = 0; kk < kTok / 16; ++kk)
                             umma_ss(tmem + kColO + 32 * j,
                                     sdesc_sw128(slot_addr(i, j) + kk * 16 * 128, kPanelBytes, 1024),
-                                    sdesc_sw128(pb + Smem::kPT + kk * 32, 16, 1024), idesc_o, 1u);
+                                    sdesc_sw128(pb + kk * 32, 16, 1024), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+                        if (rem) {
+#pragma unroll
+                            for (int kk = 0; kk < kTok / 16; ++kk)
+                                umma_ss(tmem + kColO + 32 * j,
+                                        sdesc_sw128(slot_addr(i, j) + kk * 16 * 128, kPanelBytes, 1024),
+                                        sdesc_sw128(pb + Smem::kPT + kk * 32, 16, 1024), idesc_o, 1u);
+                        }
+                        umma_commit(&empty[(i * kPairs + j) % kSlots]);
                     }
-                    umma_commit(&empty[(i * kPairs + j) % kSlots]);
+                    umma_commit(&pvdone[i & 1]);
                 }
-                umma_commit(&pvdone[i & 1]);
-            };
-            ok = mbar_wait(qready, 0, abort_flag, p.status);
-            if (ok) tc_fence_after();
-            // Issue S(nq) once its stage has landed and S(nq - 2) was read, and O(np) once its P^T is
-            // written -- whichever is ready first, so that a stage still in flight does not hold back
-            // the products (and the ring slots they free) of one that is done.  Gives up like
-            // mbar_wait when nothing moves.
-            int nq = 0, np = 0, pairs_in = 0;
-            uint32_t idle = 0;
-            unsigned long long t_idle = 0;
-            while (ok && np < n_stages) {
-                bool moved = false;
-                if (np < nq && mbar_test(&pfull[np & 1], (np >> 1) & 1)) {
-                    tc_fence_after();
-                    issue_o(np);
-                    ++np;
-                    moved = true;
-                }
-                if (nq < n_stages && (nq < 2 || mbar_test(&sfree[nq & 1], ((nq - 2) >> 1) & 1))) {
-                    while (pairs_in < kPairs) {
-                        const int n = nq * kPairs + pairs_in;
-                        if (!mbar_test(&full[n % kSlots], (n / kSlots) & 1)) break;
-                        ++pairs_in;
-                    }
-                    if (pairs_in == kPairs) {
-                        tc_fence_after();
-                        issue_s(nq);
-                        ++nq;
-                        pairs_in = 0;
-                        moved = true;
-                    }
-                }
-                if (moved) {
-                    idle = 0;
-                } else if (++idle == 1) {
-                    t_idle = global_ns();
-                } else if ((idle & 63u) == 0) {
-                    if (*abort_flag) {
-                        ok = false;
-                    } else if (global_ns() - t_idle > kWaitLimitNs) {
-                        record_timeout(p.status);
-                        *abort_flag = 1;
-                        ok = false;
-                    }
-                }
+                umma_commit(ok ? odone : drain_o);
+                if (!ok) mbar_wait_drain(drain_o, 0, p.status);
             }
-            umma_commit(ok ? odone : drain);
-            if (!ok) mbar_wait_drain(drain, 0, p.status);
         }
         __syncwarp();
     } else {
