@@ -509,7 +509,12 @@ bool mla_ws_prefers_tc(int B, int h, long long cache_rows, int sms) {
     return mla_warp_level_ctas(B, h, sms) < sms && cache_rows >= kMlaWsMinAvgRows * B;
 }
 
-size_t mla_ws_bytes(int B, int h, int sms) { return mla_tc_workspace_bytes(B, h, sms); }
+// The workspace a shape needs: none where the tensor-core kernel can never be picked
+// (16 heads or fewer, or this kernel already filling the SMs), whatever the lengths.
+size_t mla_ws_bytes(int B, int h, int sms) {
+    if (h <= kMlaHeads || mla_warp_level_ctas(B, h, sms) >= sms) return 0;
+    return mla_tc_workspace_bytes(B, h, sms);
+}
 
 int launch_mla_decode(const void *q, const void *c_kv, const int32_t *seqlens, void *out, int B, int h, float scale,
                       long long cache_rows, bool rows_known, cudaStream_t stream) {

@@ -339,11 +339,13 @@ int gqa_mla_decode_split(const void *q_absorbed, const void *c_kv, int64_t cache
                          int B, int h, int d_c, float scale,
                          void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
-/* Bytes of workspace gqa_mla_decode_split needs on the current device (the
- * tensor-core kernel's partials: ceil(h / 32) * B * splits * (32 * 512 + 64)
- * floats, with splits = max(1, min(256, SMs / (ceil(h / 32) * B)))); 0 for
- * sizes it refuses (B <= 0 or > 65535, h <= 0 or > 65535 * 16, d_c != 512).
- * Host-only. */
+/* Bytes of workspace gqa_mla_decode_split needs on the current device: the
+ * tensor-core kernel's partials, ceil(h / 32) * B * splits * (32 * 512 + 64)
+ * floats with splits = max(1, min(256, SMs / (ceil(h / 32) * B))), for shapes
+ * where that kernel can be picked (h > 16 and the warp-level kernel's CTAs
+ * fewer than the SMs); 0 for the other shapes (any non-null, aligned
+ * workspace pointer then does) and for sizes the call refuses (B <= 0 or
+ * > 65535, h <= 0 or > 65535 * 16, d_c != 512).  Host-only. */
 size_t gqa_mla_decode_split_workspace_bytes(int B, int h, int d_c);
 
 /* Which kernel runs for a shape on the current device: gqa_mla_decode_rows

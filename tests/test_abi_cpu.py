@@ -243,10 +243,11 @@ def test_mla_decode_path_rule(L, B, h, d_c, rows, want, want_ws):
 
 
 @pytest.mark.parametrize("B,h,d_c,want", [
-    (16, 32, 512, 16 * 9 * 65792),     # nine splits per sequence
+    (8, 32, 512, 8 * 18 * 65792),      # eighteen splits per sequence
     (1, 32, 512, 148 * 65792),         # one sequence over every SM
-    (300, 32, 512, 300 * 65792),       # one split each
     (2, 80, 512, 6 * 24 * 65792),      # three 32-head groups
+    (16, 32, 512, 0),                  # the warp-level kernel fills the SMs: never the tensor cores
+    (300, 32, 512, 0), (4, 16, 512, 0),
     (0, 32, 512, 0), (70000, 32, 512, 0), (1, 0, 512, 0), (1, 32, 256, 0),
 ], ids=str)
 def test_mla_split_workspace_bytes(L, B, h, d_c, want):
