@@ -25,11 +25,17 @@
 // stage's products are done.  Sequences of at most kSplitAllBelow tokens also
 // send the weights' bf16 remainders through a second product.
 //
+// Two warps issue the MMAs, one the score products and one the O^T products,
+// each committing only its own, so that O^T(i) issues as soon as its weights
+// are written.
+//
 // Ring: twelve 16 KB slots, each 64 tokens x 128 latent dims (two 64-dim
 // panels of 128-byte swizzled rows, one M block of O^T): three stages.  One
 // CTA per SM (shared memory and all of TMEM).  The splits of one (sequence,
-// 32-head group) form a cluster and merge through distributed shared memory.
-// No global scratch.  Every wait is bounded.
+// 32-head group) either form a cluster (at most 16) and merge through
+// distributed shared memory, or, given a workspace, write their partial
+// results there for a second launch to merge (any number of splits).  Every
+// wait is bounded.
 #include <cooperative_groups.h>
 
 #include <algorithm>
