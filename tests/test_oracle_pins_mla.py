@@ -10,7 +10,10 @@ the latent c itself.  Pinned here:
     an integer, so attention over the explicit keys K = c W^T (values c) and the
     absorbed decode over c with q' = q W give identical fp64 results;
   - one cached token returns that latent row exactly;
-  - the default scale is d_c ** -0.5 (the factor in that page's code).
+  - the default scale is d_c ** -0.5 (the factor in that page's code);
+  - two tokens: the logistic closed form of a two-way softmax;
+  - the softmax is over a set (row order within a sequence does not matter) and
+    sequences do not see one another's rows.
 """
 import numpy as np
 import torch
@@ -56,3 +59,38 @@ def test_single_token_returns_the_latent():
 def test_default_scale_is_latent_dim():
     q, c, lens = inputs.mla_decode_inputs(3, 2, 4, 16, [5, 9])
     assert np.array_equal(oracle.mla_decode(q, c, lens), oracle.mla_decode(q, c, lens, scale=16 ** -0.5))
+
+
+def test_two_tokens_follow_the_logistic_closed_form():
+    """Two cached tokens: the weight of the first is the logistic function of the score
+    difference, sigma((q'.c0 - q'.c1) * scale), and the output mixes the two latents."""
+    q, c, lens = inputs.mla_decode_inputs(4, 1, 3, 8, 2)
+    scale = 0.25
+    got = oracle.mla_decode(q, c, lens, scale=scale)
+    qd, cd = q.double().numpy()[0], c.double().numpy()
+    for i in range(3):
+        delta = (qd[i] @ cd[0] - qd[i] @ cd[1]) * scale
+        w0 = 1.0 / (1.0 + np.exp(-delta))
+        np.testing.assert_allclose(got[0, i], w0 * cd[0] + (1.0 - w0) * cd[1], rtol=0, atol=1e-12)
+
+
+def test_token_order_does_not_matter():
+    """The softmax runs over a set: permuting a sequence's cached rows leaves its output."""
+    lens = torch.tensor([9, 5], dtype=torch.int32)
+    q, c, lens = inputs.mla_decode_inputs(6, 2, 4, 16, lens)
+    perm = torch.cat([torch.randperm(9, generator=torch.Generator().manual_seed(1)),
+                      9 + torch.randperm(5, generator=torch.Generator().manual_seed(2))])
+    np.testing.assert_allclose(oracle.mla_decode(q, c[perm], lens), oracle.mla_decode(q, c, lens), rtol=0, atol=1e-12)
+
+
+def test_sequences_are_independent():
+    """Each sequence's output depends only on its own rows: the batch equals each sequence alone."""
+    lens = torch.tensor([3, 0, 6, 1], dtype=torch.int32)
+    q, c, lens = inputs.mla_decode_inputs(7, 4, 2, 8, lens)
+    got = oracle.mla_decode(q, c, lens)
+    off = 0
+    for b in range(4):
+        n = int(lens[b])
+        alone = oracle.mla_decode(q[b:b + 1], c[off:off + n], lens[b:b + 1])
+        np.testing.assert_allclose(got[b:b + 1], alone, rtol=0, atol=1e-13)
+        off += n
