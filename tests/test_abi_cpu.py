@@ -252,3 +252,25 @@ def test_mla_decode_path_rule(L, B, h, d_c, rows, want, want_ws):
 ], ids=str)
 def test_mla_split_workspace_bytes(L, B, h, d_c, want):
     assert L.gqa_mla_decode_split_workspace_bytes(B, h, d_c) == want
+
+
+W256 = 1 << 20   # a 256-byte aligned stand-in workspace address (never dereferenced: these calls return first)
+
+
+@pytest.mark.parametrize("args,ws,ws_bytes,expect", [
+    # q_absorbed, c_kv, cache_rows, seqlens, out, B, h, d_c, scale
+    ((0, A, 100, A, A, 2, 32, 512, 0.04), W256, 1 << 30, _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, 100, A + 1, A, 2, 32, 512, 0.04), W256, 1 << 30, _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, -1, A, A, 2, 32, 512, 0.04), W256, 1 << 30, _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, 100, A, A, 0, 32, 512, 0.04), W256, 1 << 30, _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, 100, A, A, 70000, 32, 512, 0.04), W256, 1 << 30, _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, 100, A, A, 2, 0, 512, 0.04), W256, 1 << 30, _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, 100, A, A, 2, 32, 512, -1.0), W256, 1 << 30, _lib.GQA_ERR_INVALID_ARG),
+    ((A, A, 100, A, A, 2, 32, 256, 0.04), W256, 1 << 30, _lib.GQA_ERR_UNSUPPORTED),
+    ((A, A, 100, A, A, 2, 32, 512, 0.04), 0, 1 << 30, _lib.GQA_ERR_INVALID_ARG),            # no workspace
+    ((A, A, 100, A, A, 2, 32, 512, 0.04), W256 + 16, 1 << 30, _lib.GQA_ERR_INVALID_ARG),    # misaligned
+    ((A, A, 20000, A, A, 2, 32, 512, 0.04), W256, 1000, _lib.GQA_ERR_INVALID_ARG),          # too small
+])
+def test_mla_decode_split_rejects(L, args, ws, ws_bytes, expect):
+    """gqa_mla_decode_split's argument and workspace checks (all before any launch)."""
+    assert gqa.gqa_mla_decode_split(*args, ws, ws_bytes, None) == expect
