@@ -164,7 +164,7 @@ size_t gqa_decode_split_workspace_bytes(int B, int h, int n_kv, int d_h);
  * instance a plug-in running inside another framework that must not touch
  * that framework's memory pool, or a serving loop that forbids allocations
  * once it has started (cudaMalloc synchronises the device and fails when the
- * memory is fully reserved).  The paper has no counterpart: this is an
+ * memory is fully reserved).  The pages describe no such call: this is an
  * interface convenience, not part of the method.
  *   Same arguments and result as gqa_decode_split, without the workspace:
  *   the workspace is a fixed 16 MiB array inside the library, which every

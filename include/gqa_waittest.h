@@ -12,7 +12,7 @@
  * memory and returns, and the context stays usable.  Every other entry point
  * of include/gqa.h is exported unchanged.
  *
- * The paper has no counterpart: this exists only to exercise the bounded
+ * The pages describe no such call: this exists only to exercise the bounded
  * waits.
  */
 #ifndef GQA_B200_WAITTEST_H
