@@ -468,7 +468,7 @@ def mla_leg(args, device, world, w=None):
     if gqa.gqa_get_device_status() != 0:
         raise RuntimeError("device status after the MLA decode leg")
     return {"kv_bytes": nbytes, "kernel_ms": kern_ms, "steps": steps, "copies": copies, "workload": w.name,
-            "B": w.B, "path": gqa.gqa_mla_decode_path(w.B, w.h, w.d, int(lens.clamp(min=0).sum()))}
+            "B": w.B, "path": gqa.gqa_mla_decode_path(w.B, w.h, w.d, int(lens.clamp(min=0).sum()), 1)}
 
 
 def prefill_leg(args, device, world):
@@ -607,7 +607,8 @@ def main():
         line[key] = {
             "metric": "MLA decode latent-cache GB/s", "workload": r["workload"], "value": world * gbs,
             "unit": "GB/s", "ms_per_call": r["kernel_ms"], "steps": r["steps"],
-            "kernel": ["warp-level MMA", "tcgen05"][r["path"]],
+            "kernel": {0: "warp-level MMA", 1: "tcgen05, splits merged in a cluster",
+                       2: "tcgen05, splits merged through a workspace"}.get(r["path"], "unknown"),
             "tokens_per_s": world * r["B"] / (r["kernel_ms"] / 1e3), "l2": f"{r['copies']} cache copies rotated",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s", "frac": gbs / pk["hbm"],
                          "traffic": kernel_traffic(tk),
